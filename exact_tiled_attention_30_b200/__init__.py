@@ -1,0 +1,183 @@
+"""Exact tiled attention (FlashAttention-2 method) for B200 / sm_100a.
+
+Thin Python binding of the C ABI declared in ``include/fa2.h``: every function
+with an ``fa2_`` name marshals its arguments (device pointers, sizes, the
+current CUDA stream) and calls the entry point of the same name in
+``libfa2_b200.so``. All arithmetic runs in that library's CUDA kernels; there is
+no fallback. If the library is missing the import fails loudly; build it with
+``python -m exact_tiled_attention_30_b200.build``.
+
+``attention_forward`` / ``attention_backward`` are conveniences that allocate
+the outputs (and the backward workspace) with PyTorch and then call the C ABI.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "FA2Error", "LIB_PATH", "load_library", "fa2_forward", "fa2_backward", "fa2_backward_workspace_size",
+    "fa2_status_string", "fa2_get_device_status", "fa2_clear_device_status",
+    "attention_forward", "attention_backward", "STATUS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa2_b200.so")
+
+STATUS = {0: "FA2_OK", 1: "FA2_ERR_INVALID_ARG", 2: "FA2_ERR_UNSUPPORTED",
+          3: "FA2_ERR_MISALIGNED", 4: "FA2_ERR_CUDA", 5: "FA2_ERR_TIMEOUT"}
+
+
+class FA2Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library():
+    """The ctypes handle of libfa2_b200.so. Raises if the library was not built:
+    there is no CPU or PyTorch fallback for any entry point."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: the CUDA library must be built "
+            "(python -m exact_tiled_attention_30_b200.build); there is no CPU fallback")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.fa2_forward.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, ctypes.c_float, vp]
+    lib.fa2_forward.restype = i
+    lib.fa2_backward_workspace_size.argtypes = [i, i, i, i]
+    lib.fa2_backward_workspace_size.restype = ctypes.c_size_t
+    lib.fa2_backward.argtypes = [vp] * 9 + [i, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t, vp]
+    lib.fa2_backward.restype = i
+    lib.fa2_status_string.argtypes = [i]
+    lib.fa2_status_string.restype = ctypes.c_char_p
+    lib.fa2_get_device_status.argtypes = [vp, ctypes.POINTER(i)]
+    lib.fa2_get_device_status.restype = i
+    lib.fa2_clear_device_status.argtypes = []
+    lib.fa2_clear_device_status.restype = i
+    _lib = lib
+    return lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise FA2Error(fn, status)
+
+
+def _bhnd(q):
+    if q.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def _require(t, name, dtype=None):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+
+
+def fa2_forward(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """C ABI fa2_forward on torch tensors: q, k, v, o bf16 [B,H,N,d]; lse fp32 [B,H,N]."""
+    import torch
+
+    B, H, N, d = _bhnd(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _require(t, n, torch.bfloat16)
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
+    _require(lse, "lse", torch.float32)
+    if tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be [B, H, N]")
+    _check("fa2_forward", load_library().fa2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N,
+                                          d, int(bool(causal)), float(scale), _stream(stream)))
+
+
+def fa2_backward_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().fa2_backward_workspace_size(B, H, N, d))
+
+
+def fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float, workspace,
+                 stream=None) -> None:
+    """C ABI fa2_backward on torch tensors; workspace is a uint8 CUDA tensor."""
+    import torch
+
+    B, H, N, d = _bhnd(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _require(t, n, torch.bfloat16)
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
+    _require(lse, "lse", torch.float32)
+    _require(workspace, "workspace")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check("fa2_backward", load_library().fa2_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, H, N, d, int(bool(causal)), float(scale), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def fa2_status_string(status: int) -> str:
+    return load_library().fa2_status_string(int(status)).decode()
+
+
+def fa2_get_device_status(stream=None):
+    """(status, site) after synchronising the stream; status 5 = a kernel timed out."""
+    info = ctypes.c_int(0)
+    st = load_library().fa2_get_device_status(_stream(stream), ctypes.byref(info))
+    return int(st), int(info.value)
+
+
+def fa2_clear_device_status() -> None:
+    _check("fa2_clear_device_status", load_library().fa2_clear_device_status())
+
+
+def attention_forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Allocates o and lse, runs fa2_forward, returns (o, lse)."""
+    import torch
+
+    B, H, N, d = _bhnd(q)
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa2_forward(q, k, v, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+                       stream=None, workspace=None):
+    """Allocates dq, dk, dv (and the workspace unless given), runs fa2_backward."""
+    import torch
+
+    B, H, N, d = _bhnd(q)
+    if scale is None:
+        scale = d ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(fa2_backward_workspace_size(B, H, N, d), dtype=torch.uint8,
+                                device=q.device)
+    fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, stream)
+    return dq, dk, dv

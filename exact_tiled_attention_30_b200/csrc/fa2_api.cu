@@ -1,0 +1,216 @@
+// C ABI of the exact tiled attention library (declared in include/fa2.h).
+//
+// Host side only: argument checks, Tensor Memory Accelerator descriptors,
+// kernel selection and launch on the caller's stream. Every kernel of the
+// library is compiled into this one translation unit so that they share the
+// device status word.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa2.h"
+#include "sm100_ptx.cuh"
+#include "fwd_sm100.cuh"
+
+namespace {
+
+using fa2::FwdCfg;
+
+constexpr int kMaxDevices = 64;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a contiguous bf16 [BH, N, d] array seen as 3-D (d, N, BH),
+// box = 64 elements of d x box_rows rows x 1 head, 128-byte swizzle. Rows past
+// N read as zeros.
+bool make_map_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Current device must be compute capability 10.0 (B200 class, sm_100a code).
+fa2_status check_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  static int cc[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return FA2_ERR_UNSUPPORTED;
+  if (cc[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA2_ERR_CUDA;
+    }
+    cc[dev] = major * 10 + minor;
+  }
+  if (cc[dev] != 100) return FA2_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  return FA2_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa2_status check_common(int B, int H, int N, int d, float scale) {
+  if (B < 1 || H < 1 || N < 1) return FA2_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA2_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA2_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return FA2_ERR_UNSUPPORTED;
+  // every tensor index must fit the 32-bit TMA coordinates and our size_t math
+  if (static_cast<long long>(N) > (1LL << 30)) return FA2_ERR_UNSUPPORTED;
+  return FA2_OK;
+}
+
+template <class KernelT>
+fa2_status ensure_smem(KernelT kernel, int bytes, int dev, bool* done) {
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return FA2_ERR_CUDA;
+    }
+    done[dev] = true;
+  }
+  return FA2_OK;
+}
+
+template <int D>
+fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int H, int N, int causal, float scale, cudaStream_t stream, int dev) {
+  using C = FwdCfg<D>;
+  static bool smem_set[kMaxDevices] = {false};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    fa2_status st = ensure_smem(fa2::fa2_fwd_kernel<D>, C::SMEM_ALLOC, dev, smem_set);
+    if (st != FA2_OK) return st;
+  }
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv;
+  if (!make_map_bhnd(&tq, q, BH, N, D, 128) || !make_map_bhnd(&tk, k, BH, N, D, 128) ||
+      !make_map_bhnd(&tv, v, BH, N, D, 128))
+    return FA2_ERR_CUDA;
+  fa2::FwdParams p;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.H = H;
+  p.n_qtiles = (N + C::BM - 1) / C::BM;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  dim3 grid(p.n_qtiles, BH);
+  fa2::fa2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+  return FA2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa2_status_string(int status) {
+  switch (status) {
+    case FA2_OK: return "FA2_OK";
+    case FA2_ERR_INVALID_ARG: return "FA2_ERR_INVALID_ARG";
+    case FA2_ERR_UNSUPPORTED: return "FA2_ERR_UNSUPPORTED";
+    case FA2_ERR_MISALIGNED: return "FA2_ERR_MISALIGNED";
+    case FA2_ERR_CUDA: return "FA2_ERR_CUDA";
+    case FA2_ERR_TIMEOUT: return "FA2_ERR_TIMEOUT";
+    default: return "FA2_ERR_UNKNOWN";
+  }
+}
+
+fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int N, int d, int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_common(B, H, N, d, scale);
+  if (st != FA2_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA2_ERR_MISALIGNED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_forward<64>(q, k, v, o, lse, B, H, N, causal, scale, s, dev);
+  return launch_forward<128>(q, k, v, o, lse, B, H, N, causal, scale, s, dev);
+}
+
+size_t fa2_backward_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  const size_t np = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t bh = static_cast<size_t>(B) * H;
+  return bh * np * d * 4 + 2 * bh * np * 4;
+}
+
+fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                        int H, int N, int d, int causal, float scale, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace)
+    return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_common(B, H, N, d, scale);
+  if (st != FA2_OK) return st;
+  if (workspace_bytes < fa2_backward_workspace_size(B, H, N, d)) return FA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return FA2_ERR_MISALIGNED;
+  (void)causal;
+  (void)stream;
+  return FA2_ERR_UNSUPPORTED;
+}
+
+fa2_status fa2_get_device_status(void* stream, int* info) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, fa2::g_status, sizeof(word)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  if (info) *info = static_cast<int>(word & 0xFFFFu);
+  return (word & fa2::kStatusTimeout) ? FA2_ERR_TIMEOUT : FA2_OK;
+}
+
+fa2_status fa2_clear_device_status(void) {
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(fa2::g_status, &zero, sizeof(zero)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  return FA2_OK;
+}
+
+}  // extern "C"

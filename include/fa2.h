@@ -1,0 +1,114 @@
+/*
+ * fa2.h -- C ABI of the B200 (sm_100a) exact tiled attention library.
+ *
+ * The operation is exact scaled-dot-product attention, forward and backward,
+ * computed tile by tile so that the N x N score matrix never goes to HBM:
+ *   "FlashAttention (v2)" glossary page, definition paragraph (tiles held in
+ *   on-chip memory, the full score matrix never written to HBM, the result not
+ *   approximated) and results paragraph (output matches standard attention);
+ *   "FlashAttention-2" summary page, How It Works items 1-2 (work split along
+ *   the sequence as well as batch and heads; scaling done once at the end);
+ *   "FlashAttention-2: Faster Attention with Better Parallelism and Work
+ *   Partitioning" reproduction page, closing paragraph (blocks wholly above the
+ *   causal diagonal skipped, one square block per row masked elementwise) and
+ *   Figures 5-6 (forward and backward attention are the benchmarked passes).
+ *
+ * For each head (b, h) and rows i, keys j in [0, N):
+ *   S = scale * Q K^T (causal: S_ij = -inf for j > i),  P = softmax_rows(S),
+ *   O = P V,  LSE_i = ln sum_j exp(S_ij)  (natural log).
+ * Backward, for an upstream gradient dO:
+ *   D_i = sum_c dO_ic O_ic,  dP = dO V^T,  dS = P o (dP - D),
+ *   dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO.
+ *
+ * Conventions shared by every call:
+ *  - Tensors q, k, v, o, dO, dq, dk, dv are bf16, contiguous [B, H, N, d]
+ *    (row-major; d innermost). Q and K/V have the same length N
+ *    (self-attention). lse is fp32 [B, H, N].
+ *  - d must be 64 or 128. N >= 1 (any N; the last tile is masked).
+ *    B >= 1, H >= 1, B * H <= 65535.
+ *  - scale must be finite and >= 0 (typically 1/sqrt(d)).
+ *  - All pointers are device pointers (HBM), 16-byte aligned (the kernels load
+ *    tiles with the Tensor Memory Accelerator, which requires it).
+ *  - The caller owns every buffer, including the backward workspace. The
+ *    library never allocates or frees device memory and never synchronises the
+ *    stream (fa2_get_device_status is the one exception, documented there).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *    means the legacy default stream). Arguments are checked on the host before
+ *    any launch; on any error nothing is launched and nothing is written.
+ */
+#ifndef FA2_B200_H_
+#define FA2_B200_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FA2_API __attribute__((visibility("default")))
+#else
+#define FA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA2_OK = 0,
+  FA2_ERR_INVALID_ARG = 1, /* null pointer, N/B/H < 1, bad scale, workspace too small */
+  FA2_ERR_UNSUPPORTED = 2, /* d not in {64, 128}, B*H > 65535, or no sm_100 device */
+  FA2_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
+  FA2_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor map) */
+  FA2_ERR_TIMEOUT = 5      /* a kernel gave up on a bounded wait (see fa2_get_device_status) */
+} fa2_status;
+
+/*
+ * Forward pass: o = softmax(scale * q k^T [causal]) v and lse (natural log).
+ * q, k, v: inputs [B,H,N,d] bf16. o: output [B,H,N,d] bf16. lse: output
+ * [B,H,N] fp32, kept for the backward pass. causal: 0 or 1 (j <= i allowed).
+ * One kernel launch on `stream`; the grid runs over (query block, batch*head).
+ */
+FA2_API fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * Bytes of device workspace fa2_backward needs for these sizes: an fp32 dQ
+ * accumulator [B,H,Np,d] plus two fp32 row vectors [B,H,Np] (D = rowsum(dO o O)
+ * and the log2-scaled LSE), with Np = N rounded up to 128. Returns 0 for
+ * invalid sizes.
+ */
+FA2_API size_t fa2_backward_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass. Inputs q, k, v, o (the forward output), lse (the forward
+ * LSE), dO (gradient of the loss w.r.t. o). Outputs dq, dk, dv [B,H,N,d] bf16.
+ * o and lse must come from fa2_forward on the same q, k, v, causal and scale;
+ * they are trusted as given. workspace: caller-owned device memory of at least
+ * fa2_backward_workspace_size() bytes, 16-byte aligned; its contents on entry
+ * do not matter and on exit are unspecified. Three launches on `stream`:
+ * preprocess (D, log2 LSE, zero dQ accumulator), the key-block-parallel main
+ * kernel (dK, dV, and dQ accumulated with fp32 reductions), and the dQ
+ * conversion to bf16.
+ */
+FA2_API fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                        int B, int H, int N, int d, int causal, float scale,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static, NUL-terminated name of a status code. */
+FA2_API const char* fa2_status_string(int status);
+
+/*
+ * Synchronises `stream` and reports whether any kernel of this library on the
+ * current device gave up on a bounded wait since the last clear. Returns
+ * FA2_OK, FA2_ERR_TIMEOUT (then *info, if non-NULL, holds a site code), or
+ * FA2_ERR_CUDA if the synchronisation itself failed.
+ */
+FA2_API fa2_status fa2_get_device_status(void* stream, int* info);
+
+/* Clears the device-side status word of the current device (synchronous). */
+FA2_API fa2_status fa2_clear_device_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA2_B200_H_ */

@@ -1,0 +1,109 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load on a machine without a GPU, export every entry point
+``include/fa2.h`` declares, and reject bad arguments with the documented status
+codes before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa2.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_tiled_attention_30_b200 import build
+
+    build.build()
+    import exact_tiled_attention_30_b200 as m
+
+    return m.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FA2_API[^;(]*?\b(fa2_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    assert {"fa2_forward", "fa2_backward", "fa2_backward_workspace_size", "fa2_status_string",
+            "fa2_get_device_status", "fa2_clear_device_status"} <= set(declared_symbols())
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_library_exports_nothing_else(lib):
+    out = os.popen(f"nm -D --defined-only {lib._name}").read()
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    ours = {s for s in exported if s.startswith("fa2")}
+    assert ours == set(declared_symbols())
+
+
+def test_status_strings(lib):
+    import exact_tiled_attention_30_b200 as m
+
+    for code, name in m.STATUS.items():
+        assert m.fa2_status_string(code) == name
+    assert m.fa2_status_string(99) == "FA2_ERR_UNKNOWN"
+
+
+A = 0x10000  # aligned fake device address (never dereferenced: checks fail first)
+
+
+def fwd(lib, q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, causal=0, scale=0.125):
+    return lib.fa2_forward(q, k, v, o, lse, B, H, N, d, causal, ctypes.c_float(scale), None)
+
+
+def test_forward_rejects_bad_arguments(lib):
+    assert fwd(lib, q=None) == 1
+    assert fwd(lib, lse=None) == 1
+    assert fwd(lib, N=0) == 1
+    assert fwd(lib, B=0) == 1
+    assert fwd(lib, H=-1) == 1
+    assert fwd(lib, scale=float("nan")) == 1
+    assert fwd(lib, scale=float("inf")) == 1
+    assert fwd(lib, scale=-0.5) == 1
+    assert fwd(lib, d=96) == 2
+    assert fwd(lib, d=256) == 2
+    assert fwd(lib, B=256, H=256) == 2
+    assert fwd(lib, q=A + 8) == 3
+    assert fwd(lib, o=A + 2) == 3
+    assert fwd(lib, lse=A + 4) == 3
+
+
+def test_workspace_size(lib):
+    import exact_tiled_attention_30_b200 as m
+
+    assert m.fa2_backward_workspace_size(1, 1, 128, 64) == 128 * 64 * 4 + 2 * 128 * 4
+    assert m.fa2_backward_workspace_size(2, 3, 129, 128) == 6 * 256 * 128 * 4 + 2 * 6 * 256 * 4
+    assert m.fa2_backward_workspace_size(1, 1, 0, 64) == 0
+    assert m.fa2_backward_workspace_size(1, 1, 10, 32) == 0
+
+
+def bwd(lib, ptrs=None, B=1, H=1, N=128, d=64, scale=0.125, ws_bytes=None):
+    p = [A] * 10 if ptrs is None else ptrs
+    if ws_bytes is None:
+        ws_bytes = lib.fa2_backward_workspace_size(B, H, N, d)
+    return lib.fa2_backward(*p[:9], B, H, N, d, 0, ctypes.c_float(scale), p[9], ws_bytes, None)
+
+
+def test_backward_rejects_bad_arguments(lib):
+    for i in range(10):
+        p = [A] * 10
+        p[i] = None
+        assert bwd(lib, p) == 1, i
+    assert bwd(lib, ws_bytes=100) == 1
+    assert bwd(lib, N=0) == 1
+    assert bwd(lib, d=32) == 2
+    assert bwd(lib, scale=float("nan")) == 1
+    for i in range(10):
+        p = [A] * 10
+        p[i] = A + 4
+        assert bwd(lib, p) == 3, i
