@@ -16,6 +16,7 @@
 #include "fa2.h"
 #include "sm100_ptx.cuh"
 #include "fwd_sm100.cuh"
+#include "bwd_sm100.cuh"
 
 namespace {
 
@@ -135,6 +136,80 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   return FA2_OK;
 }
 
+template <int D>
+fa2_status launch_backward(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                           int H, int N, int causal, float scale, void* workspace,
+                           cudaStream_t stream, int dev) {
+  using C = fa2::BwdCfg<D>;
+  static bool smem_set[kMaxDevices] = {false};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    fa2_status st = ensure_smem(fa2::fa2_bwd_kernel<D>, C::SMEM_ALLOC, dev, smem_set);
+    if (st != FA2_OK) return st;
+  }
+  const int BH = B * H;
+  const int n_tiles = (N + 127) / 128;
+  const int Np = n_tiles * 128;
+  float* dq_acc = reinterpret_cast<float*>(workspace);
+  float* delta = dq_acc + static_cast<size_t>(BH) * Np * D;
+  float* lse2 = delta + static_cast<size_t>(BH) * Np;
+
+  fa2::BwdPreParams pp;
+  pp.o = reinterpret_cast<const __nv_bfloat16*>(o);
+  pp.dout = reinterpret_cast<const __nv_bfloat16*>(dO);
+  pp.lse = lse;
+  pp.dq_acc = dq_acc;
+  pp.delta = delta;
+  pp.lse2 = lse2;
+  pp.N = N;
+  pp.Np = Np;
+  pp.rows = static_cast<long long>(BH) * Np;
+  {
+    constexpr int rpb = 256 / (D / 8);
+    const long long want = (pp.rows + rpb - 1) / rpb;
+    const int blocks = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);
+    fa2::fa2_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(pp);
+    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+  }
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map_bhnd(&tq, q, BH, N, D, 128) || !make_map_bhnd(&tk, k, BH, N, D, 128) ||
+      !make_map_bhnd(&tv, v, BH, N, D, 128) || !make_map_bhnd(&tdo, dO, BH, N, D, 128))
+    return FA2_ERR_CUDA;
+  fa2::BwdParams bp;
+  bp.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  bp.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  bp.dq_acc = dq_acc;
+  bp.lse2 = lse2;
+  bp.delta = delta;
+  bp.N = N;
+  bp.Np = Np;
+  bp.n_ktiles = n_tiles;
+  bp.causal = causal ? 1 : 0;
+  bp.scale = scale;
+  bp.scale_log2 = scale * 1.4426950408889634f;
+  fa2::fa2_bwd_kernel<D><<<dim3(n_tiles, BH), C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, bp);
+  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+
+  fa2::BwdConvertParams cp;
+  cp.dq_acc = dq_acc;
+  cp.dq = reinterpret_cast<__nv_bfloat16*>(dq);
+  cp.N = N;
+  cp.Np = Np;
+  cp.d = D;
+  cp.total8 = static_cast<long long>(BH) * N * D / 8;
+  cp.scale = scale;
+  {
+    const long long want = (cp.total8 + 255) / 256;
+    const int blocks = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);
+    fa2::fa2_bwd_dq_convert_kernel<<<blocks, 256, 0, stream>>>(cp);
+    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+  }
+  return FA2_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -185,9 +260,13 @@ fa2_status fa2_backward(const void* q, const void* k, const void* v, const void*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
     return FA2_ERR_MISALIGNED;
-  (void)causal;
-  (void)stream;
-  return FA2_ERR_UNSUPPORTED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return launch_backward<64>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, causal, scale, workspace, s, dev);
+  return launch_backward<128>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, causal, scale, workspace, s, dev);
 }
 
 fa2_status fa2_get_device_status(void* stream, int* info) {
