@@ -17,6 +17,7 @@ import os
 
 __all__ = [
     "FA2Error", "LIB_PATH", "load_library", "fa2_forward", "fa2_backward", "fa2_backward_workspace_size",
+    "fa2_backward_preprocess", "fa2_backward_main", "fa2_backward_dq_convert",
     "fa2_status_string", "fa2_get_device_status", "fa2_clear_device_status",
     "attention_forward", "attention_backward", "STATUS",
 ]
@@ -54,6 +55,13 @@ def load_library():
     lib.fa2_backward_workspace_size.restype = ctypes.c_size_t
     lib.fa2_backward.argtypes = [vp] * 9 + [i, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t, vp]
     lib.fa2_backward.restype = i
+    lib.fa2_backward_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp, ctypes.c_size_t, vp]
+    lib.fa2_backward_preprocess.restype = i
+    lib.fa2_backward_main.argtypes = [vp] * 6 + [i, i, i, i, i, ctypes.c_float, vp,
+                                                 ctypes.c_size_t, vp]
+    lib.fa2_backward_main.restype = i
+    lib.fa2_backward_dq_convert.argtypes = [vp, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t, vp]
+    lib.fa2_backward_dq_convert.restype = i
     lib.fa2_status_string.argtypes = [i]
     lib.fa2_status_string.restype = ctypes.c_char_p
     lib.fa2_get_device_status.argtypes = [vp, ctypes.POINTER(i)]
@@ -137,6 +145,34 @@ def fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float, 
     _check("fa2_backward", load_library().fa2_backward(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
         B, H, N, d, int(bool(causal)), float(scale), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def fa2_backward_preprocess(o, lse, dout, workspace, stream=None) -> None:
+    """C ABI fa2_backward_preprocess (first of the three backward stages)."""
+    B, H, N, d = _bhnd(o)
+    _check("fa2_backward_preprocess", load_library().fa2_backward_preprocess(
+        _ptr(o), _ptr(lse), _ptr(dout), B, H, N, d, _ptr(workspace), _nbytes(workspace),
+        _stream(stream)))
+
+
+def fa2_backward_main(q, k, v, dout, dk, dv, causal: bool, scale: float, workspace,
+                      stream=None) -> None:
+    """C ABI fa2_backward_main (dK, dV and the fp32 dQ accumulator)."""
+    B, H, N, d = _bhnd(q)
+    _check("fa2_backward_main", load_library().fa2_backward_main(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)),
+        float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def fa2_backward_dq_convert(dq, scale: float, workspace, stream=None) -> None:
+    """C ABI fa2_backward_dq_convert (dq = bf16(scale * accumulator))."""
+    B, H, N, d = _bhnd(dq)
+    _check("fa2_backward_dq_convert", load_library().fa2_backward_dq_convert(
+        _ptr(dq), B, H, N, d, float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def fa2_status_string(status: int) -> str:

@@ -136,10 +136,48 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   return FA2_OK;
 }
 
+struct WsLayout {
+  float* dq_acc;
+  float* delta;
+  float* lse2;
+  int Np;
+};
+
+WsLayout ws_layout(void* workspace, int BH, int N, int d) {
+  WsLayout w;
+  w.Np = (N + 127) / 128 * 128;
+  w.dq_acc = reinterpret_cast<float*>(workspace);
+  w.delta = w.dq_acc + static_cast<size_t>(BH) * w.Np * d;
+  w.lse2 = w.delta + static_cast<size_t>(BH) * w.Np;
+  return w;
+}
+
+inline int grid_cap(long long want) {
+  return static_cast<int>(want < 148LL * 16 ? (want > 0 ? want : 1) : 148LL * 16);
+}
+
 template <int D>
-fa2_status launch_backward(const void* q, const void* k, const void* v, const void* o,
-                           const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
-                           int H, int N, int causal, float scale, void* workspace,
+fa2_status launch_bwd_pre(const void* o, const float* lse, const void* dO, int BH, int N,
+                          void* workspace, cudaStream_t stream) {
+  const WsLayout w = ws_layout(workspace, BH, N, D);
+  fa2::BwdPreParams pp;
+  pp.o = reinterpret_cast<const __nv_bfloat16*>(o);
+  pp.dout = reinterpret_cast<const __nv_bfloat16*>(dO);
+  pp.lse = lse;
+  pp.dq_acc = w.dq_acc;
+  pp.delta = w.delta;
+  pp.lse2 = w.lse2;
+  pp.N = N;
+  pp.Np = w.Np;
+  pp.rows = static_cast<long long>(BH) * w.Np;
+  constexpr int rpb = 256 / (D / 8);
+  fa2::fa2_bwd_pre_kernel<D><<<grid_cap((pp.rows + rpb - 1) / rpb), 256, 0, stream>>>(pp);
+  return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
+}
+
+template <int D>
+fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                           void* dv, int BH, int N, int causal, float scale, void* workspace,
                            cudaStream_t stream, int dev) {
   using C = fa2::BwdCfg<D>;
   static bool smem_set[kMaxDevices] = {false};
@@ -149,31 +187,7 @@ fa2_status launch_backward(const void* q, const void* k, const void* v, const vo
     fa2_status st = ensure_smem(fa2::fa2_bwd_kernel<D>, C::SMEM_ALLOC, dev, smem_set);
     if (st != FA2_OK) return st;
   }
-  const int BH = B * H;
-  const int n_tiles = (N + 127) / 128;
-  const int Np = n_tiles * 128;
-  float* dq_acc = reinterpret_cast<float*>(workspace);
-  float* delta = dq_acc + static_cast<size_t>(BH) * Np * D;
-  float* lse2 = delta + static_cast<size_t>(BH) * Np;
-
-  fa2::BwdPreParams pp;
-  pp.o = reinterpret_cast<const __nv_bfloat16*>(o);
-  pp.dout = reinterpret_cast<const __nv_bfloat16*>(dO);
-  pp.lse = lse;
-  pp.dq_acc = dq_acc;
-  pp.delta = delta;
-  pp.lse2 = lse2;
-  pp.N = N;
-  pp.Np = Np;
-  pp.rows = static_cast<long long>(BH) * Np;
-  {
-    constexpr int rpb = 256 / (D / 8);
-    const long long want = (pp.rows + rpb - 1) / rpb;
-    const int blocks = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);
-    fa2::fa2_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(pp);
-    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
-  }
-
+  const WsLayout w = ws_layout(workspace, BH, N, D);
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map_bhnd(&tq, q, BH, N, D, 128) || !make_map_bhnd(&tk, k, BH, N, D, 128) ||
       !make_map_bhnd(&tv, v, BH, N, D, 128) || !make_map_bhnd(&tdo, dO, BH, N, D, 128))
@@ -181,32 +195,38 @@ fa2_status launch_backward(const void* q, const void* k, const void* v, const vo
   fa2::BwdParams bp;
   bp.dk = reinterpret_cast<__nv_bfloat16*>(dk);
   bp.dv = reinterpret_cast<__nv_bfloat16*>(dv);
-  bp.dq_acc = dq_acc;
-  bp.lse2 = lse2;
-  bp.delta = delta;
+  bp.dq_acc = w.dq_acc;
+  bp.lse2 = w.lse2;
+  bp.delta = w.delta;
   bp.N = N;
-  bp.Np = Np;
-  bp.n_ktiles = n_tiles;
+  bp.Np = w.Np;
+  bp.n_ktiles = w.Np / 128;
   bp.causal = causal ? 1 : 0;
   bp.scale = scale;
   bp.scale_log2 = scale * 1.4426950408889634f;
-  fa2::fa2_bwd_kernel<D><<<dim3(n_tiles, BH), C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, bp);
-  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+  fa2::fa2_bwd_kernel<D><<<dim3(bp.n_ktiles, BH), C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, bp);
+  return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
+}
 
+fa2_status launch_bwd_convert(void* dq, int BH, int N, int d, float scale, void* workspace,
+                              cudaStream_t stream) {
+  const WsLayout w = ws_layout(workspace, BH, N, d);
   fa2::BwdConvertParams cp;
-  cp.dq_acc = dq_acc;
+  cp.dq_acc = w.dq_acc;
   cp.dq = reinterpret_cast<__nv_bfloat16*>(dq);
   cp.N = N;
-  cp.Np = Np;
-  cp.d = D;
-  cp.total8 = static_cast<long long>(BH) * N * D / 8;
+  cp.Np = w.Np;
+  cp.d = d;
+  cp.total8 = static_cast<long long>(BH) * N * d / 8;
   cp.scale = scale;
-  {
-    const long long want = (cp.total8 + 255) / 256;
-    const int blocks = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);
-    fa2::fa2_bwd_dq_convert_kernel<<<blocks, 256, 0, stream>>>(cp);
-    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
-  }
+  fa2::fa2_bwd_dq_convert_kernel<<<grid_cap((cp.total8 + 255) / 256), 256, 0, stream>>>(cp);
+  return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
+}
+
+fa2_status check_workspace(int B, int H, int N, int d, const void* workspace, size_t bytes) {
+  if (!workspace) return FA2_ERR_INVALID_ARG;
+  if (bytes < fa2_backward_workspace_size(B, H, N, d)) return FA2_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return FA2_ERR_MISALIGNED;
   return FA2_OK;
 }
 
@@ -248,6 +268,56 @@ size_t fa2_backward_workspace_size(int B, int H, int N, int d) {
   return bh * np * d * 4 + 2 * bh * np * 4;
 }
 
+fa2_status fa2_backward_preprocess(const void* o, const float* lse, const void* dO, int B, int H,
+                                   int N, int d, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (!o || !lse || !dO) return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_common(B, H, N, d, 1.0f);
+  if (st != FA2_OK) return st;
+  st = check_workspace(B, H, N, d, workspace, workspace_bytes);
+  if (st != FA2_OK) return st;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(dO)) return FA2_ERR_MISALIGNED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd_pre<64>(o, lse, dO, B * H, N, workspace, s)
+                 : launch_bwd_pre<128>(o, lse, dO, B * H, N, workspace, s);
+}
+
+fa2_status fa2_backward_main(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                             void* dv, int B, int H, int N, int d, int causal, float scale,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dk || !dv) return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_common(B, H, N, d, scale);
+  if (st != FA2_OK) return st;
+  st = check_workspace(B, H, N, d, workspace, workspace_bytes);
+  if (st != FA2_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) ||
+      !aligned16(dv))
+    return FA2_ERR_MISALIGNED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd_main<64>(q, k, v, dO, dk, dv, B * H, N, causal, scale, workspace, s, dev)
+                 : launch_bwd_main<128>(q, k, v, dO, dk, dv, B * H, N, causal, scale, workspace, s, dev);
+}
+
+fa2_status fa2_backward_dq_convert(void* dq, int B, int H, int N, int d, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dq) return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_common(B, H, N, d, scale);
+  if (st != FA2_OK) return st;
+  st = check_workspace(B, H, N, d, workspace, workspace_bytes);
+  if (st != FA2_OK) return st;
+  if (!aligned16(dq)) return FA2_ERR_MISALIGNED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+  return launch_bwd_convert(dq, B * H, N, d, scale, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
 fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
                         const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
                         int H, int N, int d, int causal, float scale, void* workspace,
@@ -264,9 +334,16 @@ fa2_status fa2_backward(const void* q, const void* k, const void* v, const void*
   st = check_device(&dev);
   if (st != FA2_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    return launch_backward<64>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, causal, scale, workspace, s, dev);
-  return launch_backward<128>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, causal, scale, workspace, s, dev);
+  const int BH = B * H;
+  if (d == 64) {
+    st = launch_bwd_pre<64>(o, lse, dO, BH, N, workspace, s);
+    if (st == FA2_OK) st = launch_bwd_main<64>(q, k, v, dO, dk, dv, BH, N, causal, scale, workspace, s, dev);
+  } else {
+    st = launch_bwd_pre<128>(o, lse, dO, BH, N, workspace, s);
+    if (st == FA2_OK) st = launch_bwd_main<128>(q, k, v, dO, dk, dv, BH, N, causal, scale, workspace, s, dev);
+  }
+  if (st == FA2_OK) st = launch_bwd_convert(dq, BH, N, d, scale, workspace, s);
+  return st;
 }
 
 fa2_status fa2_get_device_status(void* stream, int* info) {

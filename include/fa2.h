@@ -93,6 +93,26 @@ FA2_API fa2_status fa2_backward(const void* q, const void* k, const void* v, con
                         int B, int H, int N, int d, int causal, float scale,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * The three stages fa2_backward launches, callable one at a time (same
+ * arguments and checks as fa2_backward; run them in this order on one stream,
+ * with the same workspace, to get exactly fa2_backward's result):
+ *  fa2_backward_preprocess  D = rowsum(dO o O), LSE * log2(e), dQ accumulator
+ *                           zeroed; padding rows get D = 0 and LSE = +inf.
+ *  fa2_backward_main        dK, dV (bf16 outputs) and the fp32 dQ accumulator.
+ *  fa2_backward_dq_convert  dq = bf16(scale * accumulator).
+ * Splitting them lets a caller time or overlap the stages individually.
+ */
+FA2_API fa2_status fa2_backward_preprocess(const void* o, const float* lse, const void* dO,
+                                           int B, int H, int N, int d, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+FA2_API fa2_status fa2_backward_main(const void* q, const void* k, const void* v, const void* dO,
+                                     void* dk, void* dv, int B, int H, int N, int d, int causal,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+FA2_API fa2_status fa2_backward_dq_convert(void* dq, int B, int H, int N, int d, float scale,
+                                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static, NUL-terminated name of a status code. */
 FA2_API const char* fa2_status_string(int status);
 

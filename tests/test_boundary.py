@@ -31,7 +31,8 @@ def declared_symbols():
 
 def test_header_declares_the_abi():
     assert {"fa2_forward", "fa2_backward", "fa2_backward_workspace_size", "fa2_status_string",
-            "fa2_get_device_status", "fa2_clear_device_status"} <= set(declared_symbols())
+            "fa2_get_device_status", "fa2_clear_device_status", "fa2_backward_preprocess",
+            "fa2_backward_main", "fa2_backward_dq_convert"} <= set(declared_symbols())
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -107,3 +108,20 @@ def test_backward_rejects_bad_arguments(lib):
         p = [A] * 10
         p[i] = A + 4
         assert bwd(lib, p) == 3, i
+
+
+def test_backward_stages_reject_bad_arguments(lib):
+    ws = lib.fa2_backward_workspace_size(1, 1, 128, 64)
+    f = ctypes.c_float
+    assert lib.fa2_backward_preprocess(None, A, A, 1, 1, 128, 64, A, ws, None) == 1
+    assert lib.fa2_backward_preprocess(A, A, A, 1, 1, 128, 64, None, ws, None) == 1
+    assert lib.fa2_backward_preprocess(A, A, A, 1, 1, 128, 64, A, ws - 1, None) == 1
+    assert lib.fa2_backward_preprocess(A, A, A, 1, 1, 128, 48, A, ws, None) == 2
+    assert lib.fa2_backward_preprocess(A, A + 4, A, 1, 1, 128, 64, A, ws, None) == 3
+    assert lib.fa2_backward_main(A, A, A, A, A, None, 1, 1, 128, 64, 0, f(0.1), A, ws, None) == 1
+    assert lib.fa2_backward_main(A, A, A, A, A, A, 1, 1, 128, 64, 0, f(-1.0), A, ws, None) == 1
+    assert lib.fa2_backward_main(A, A, A, A, A, A, 1, 1, 128, 64, 0, f(0.1), A + 8, ws, None) == 3
+    assert lib.fa2_backward_main(A, A, A, A + 2, A, A, 1, 1, 128, 64, 0, f(0.1), A, ws, None) == 3
+    assert lib.fa2_backward_dq_convert(None, 1, 1, 128, 64, f(0.1), A, ws, None) == 1
+    assert lib.fa2_backward_dq_convert(A, 1, 1, 128, 64, f(0.1), A, 16, None) == 1
+    assert lib.fa2_backward_dq_convert(A + 2, 1, 1, 128, 64, f(0.1), A, ws, None) == 3
