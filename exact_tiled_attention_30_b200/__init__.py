@@ -217,3 +217,22 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: float
                                 device=q.device)
     fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, stream)
     return dq, dk, dv
+
+
+def fa2_backward_noalloc(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float,
+                         stream=None) -> None:
+    """C ABI fa2_backward_noalloc: the backward pass with its scratch in a fixed
+    device array inside the library (FA2_NOALLOC_SCRATCH_BYTES = 64 MiB) instead
+    of a workspace, for callers that cannot allocate device memory at that point.
+    Raises FA2Error(FA2_ERR_UNSUPPORTED) when the sizes need more scratch than that.
+    Calls on one stream are safe; calls that overlap on the GPU race on the array."""
+    lib = load_library()
+    fn = lib.fa2_backward_noalloc
+    if fn.restype is not ctypes.c_int or fn.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        fn.argtypes = [vp] * 9 + [i, i, i, i, i, ctypes.c_float, vp]
+        fn.restype = i
+    B, H, N, d = _bhnd(q)
+    _check("fa2_backward_noalloc", fn(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, H, N, d, int(bool(causal)), float(scale), _stream(stream)))

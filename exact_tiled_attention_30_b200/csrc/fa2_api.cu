@@ -370,3 +370,77 @@ fa2_status fa2_clear_device_status(void) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory when they run the backward pass:
+// code that reserved all of its device memory up front and may not call
+// cudaMalloc afterwards, plugins whose host forbids allocation (and the
+// implicit device synchronisation cudaMalloc may cause) on its hot path, or
+// plain C callers with no allocator of their own to size a workspace with.
+// fa2_backward_noalloc serves them: its scratch (fp32 dQ accumulator, D and the
+// log2-scaled LSE) lives in the fixed device array below instead of a
+// workspace argument. Every GPU that loads this library keeps the array for
+// the life of the process.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA2_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on device `dev` (which must be current).
+// In host code the array's name only stands in for the symbol; the address a
+// kernel may use comes from cudaGetSymbolAddress, looked up once per device.
+void* noalloc_scratch(int dev, fa2_status* st) {
+  static void* addr[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      *st = FA2_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  *st = FA2_OK;
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+fa2_status fa2_backward_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                int B, int H, int N, int d, int causal, float scale,
+                                void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_common(B, H, N, d, scale);
+  if (st != FA2_OK) return st;
+  if (fa2_backward_workspace_size(B, H, N, d) > static_cast<size_t>(FA2_NOALLOC_SCRATCH_BYTES))
+    return FA2_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA2_ERR_MISALIGNED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+  void* scratch = noalloc_scratch(dev, &st);
+  if (st != FA2_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  // the preprocess kernel re-zeroes the dQ accumulator and rewrites D and LSE,
+  // so whatever an earlier call left in the array does not matter
+  if (d == 64) {
+    st = launch_bwd_pre<64>(o, lse, dO, BH, N, scratch, s);
+    if (st == FA2_OK) st = launch_bwd_main<64>(q, k, v, dO, dk, dv, BH, N, causal, scale, scratch, s, dev);
+  } else {
+    st = launch_bwd_pre<128>(o, lse, dO, BH, N, scratch, s);
+    if (st == FA2_OK) st = launch_bwd_main<128>(q, k, v, dO, dk, dv, BH, N, causal, scale, scratch, s, dev);
+  }
+  if (st == FA2_OK) st = launch_bwd_convert(dq, BH, N, d, scale, scratch, s);
+  return st;
+}
+
+}  // extern "C"

@@ -113,6 +113,37 @@ FA2_API fa2_status fa2_backward_main(const void* q, const void* k, const void* v
 FA2_API fa2_status fa2_backward_dq_convert(void* dq, int B, int H, int N, int d, float scale,
                                            void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Backward pass that allocates nothing and takes no workspace. (The paper has
+ * no counterpart; this is a deployment convenience of this library.)
+ *
+ * For callers that cannot allocate device memory when they run the backward:
+ * applications that reserve all device memory at start-up and may not call
+ * cudaMalloc later, plugins whose host forbids allocation (and the device
+ * synchronisation it can cause) on the hot path, or C callers without an
+ * allocator to size a workspace with. Same arguments, checks and results as
+ * fa2_backward, minus workspace/workspace_bytes: the scratch (fp32 dQ
+ * accumulator, D, log2-scaled LSE) lives in a fixed device array of
+ * FA2_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *  - Returns FA2_ERR_UNSUPPORTED, without launching anything, when
+ *    fa2_backward_workspace_size(B, H, N, d) > FA2_NOALLOC_SCRATCH_BYTES
+ *    (for example B*H*N*d above about 16 million elements).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls share the one array: calls whose kernels overlap on the GPU
+ *    (different streams without ordering between them) race on it and give
+ *    wrong results. Calls ordered on one stream are safe; each call
+ *    re-initialises the parts that must start at zero.
+ *  - Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+#define FA2_NOALLOC_SCRATCH_BYTES (64u << 20)
+FA2_API fa2_status fa2_backward_noalloc(const void* q, const void* k, const void* v,
+                                        const void* o, const float* lse, const void* dO,
+                                        void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                                        int causal, float scale, void* stream);
+
 /* Static, NUL-terminated name of a status code. */
 FA2_API const char* fa2_status_string(int status);
 
