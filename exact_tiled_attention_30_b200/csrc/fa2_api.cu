@@ -126,11 +126,11 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.N = N;
-  p.H = H;
   p.n_qtiles = (N + C::BM - 1) / C::BM;
+  p.n_pairs = (p.n_qtiles + 1) / 2;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
-  dim3 grid(p.n_qtiles, BH);
+  dim3 grid(p.n_pairs, BH);
   fa2::fa2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
   return FA2_OK;
@@ -444,3 +444,11 @@ fa2_status fa2_backward_noalloc(const void* q, const void* k, const void* v, con
 }
 
 }  // extern "C"
+
+#ifdef FA2_TRACE
+// Debug builds only: copies the trace stamps of the last traced launch.
+extern "C" FA2_API int fa2_debug_trace_read(unsigned long long* host, int n) {
+  if (n > 64 * 64) n = 64 * 64;
+  return cudaMemcpyFromSymbol(host, fa2::g_trace, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : 1;
+}
+#endif

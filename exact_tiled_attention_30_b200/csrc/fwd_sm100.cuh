@@ -3,25 +3,35 @@
 // Method ("FlashAttention-2" summary page, How It Works items 1-3; "FlashAttention
 // (v2)" glossary page, definition and mechanism paragraphs; reproduction page of
 // the FlashAttention-2 paper, closing paragraph on causal blocks):
-//   * one CTA per (query block of 128 rows, batch*head): the sequence itself is
-//     split across CTAs, not just batch and heads;
+//   * the sequence is split across CTAs, not just batch and heads: one CTA per
+//     (256-row query block, batch*head);
 //   * K/V tiles of 128 keys stream through shared memory; the running row max m
 //     and row sum l (online softmax) keep the N x N scores on chip;
-//   * the accumulator is rescaled only when the running max grows, and divided
-//     by l once, in the epilogue;
+//   * the accumulator is divided by l once, in the epilogue;
 //   * causal: key tiles wholly above the diagonal are never visited and only
-//     the diagonal tile is masked elementwise.
+//     the diagonal tile of each query tile is masked elementwise.
 //
 // B200 mapping (the pages' A100/H100 tiling is prior art only):
-//   warp 4       TMA producer: Q once, then K_j/V_j into a STAGES-deep ring
-//   warp 5       MMA issuer + TMEM owner: S_j = Q K_j^T (tcgen05, smem x smem ->
-//                TMEM, double-buffered), O += P_j V_j (P from TMEM, V from smem)
-//   warps 0-3    softmax: thread t owns query row t (= TMEM lane t); reads S_j
-//                with tcgen05.ld, updates m and l, rescales O in TMEM when the
-//                max grew, writes P_j as bf16 into TMEM; finally O/l and LSE.
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+D),
-// P [384,448) as bf16 pairs. Scores are kept in base 2: c = scale * log2(e)
-// folds the softmax scale into the exponent, m is stored pre-multiplied by c.
+//   warp 8        TMA producer: Q0, Q1 once, then K_j/V_j into a STAGES-deep ring
+//   warp 9        MMA issuer + TMEM owner. Per key tile j it issues
+//                 PV0_j, S0_{j+1}, PV1_j, S1_{j+1} (in that order), so while one
+//                 warpgroup runs the softmax of its tile the tensor core works on
+//                 the other tile: S_t = Q_t K_j^T (smem x smem -> TMEM) and
+//                 O_t += P_t V_j (P from TMEM, V from smem).
+//   warps 0-3     softmax of query tile 0, warps 4-7 of query tile 1: thread r
+//                 owns row r (TMEM lane r); tcgen05.ld of S, row max, exp2,
+//                 row sum, P written back as bf16 over the first 64 columns of S.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
+// O1 [256+D, 256+2D). Scores are kept in base 2: c = scale * log2(e) folds the
+// softmax scale into the exponent and m is stored pre-multiplied by c.
+//
+// Rescaling: a row's reference max m only moves when the new tile's max exceeds
+// it by more than 8 (base-2 units). Otherwise P keeps using the old m (entries
+// up to 2^8, exact in fp32 accumulation and bf16's relative precision) and O is
+// not touched. The result is unchanged because O and l share the same m and O/l
+// is formed once at the end; LSE = m + log2(l) uses that same m. O is divided
+// by the sum of the bf16-rounded weights it was accumulated with, so it stays
+// a convex combination of V rows when one weight dominates; LSE uses the fp32 sum.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -31,62 +41,68 @@ namespace fa2 {
 template <int D>
 struct FwdCfg {
   static_assert(D == 64 || D == 128, "head dim");
-  static constexpr int BM = 128;
-  static constexpr int BN = 128;
-  static constexpr int STAGES = (D == 64) ? 3 : 2;
+  static constexpr int BM = 128;                      // rows per query tile (two per CTA)
+  static constexpr int BN = 128;                      // keys per K/V tile
+  static constexpr int STAGES = (D == 64) ? 4 : 2;
   static constexpr int CHUNKS = D / 64;               // 128-byte swizzle atoms across d
   static constexpr int TILE_BYTES = BM * D * 2;       // one Q, K or V tile
   static constexpr int CHUNK_BYTES = 128 * 128;       // one [128 rows][64] bf16 box
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = TILE_BYTES;                           // + s * 2 * TILE_BYTES
-  static constexpr int OFF_V = 2 * TILE_BYTES;                       // + s * 2 * TILE_BYTES
-  static constexpr int OFF_BAR = TILE_BYTES * (1 + 2 * STAGES);
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full, o_done, drain
-  static constexpr int NUM_BARS = 1 + 2 * STAGES + 2 + 3;
+  static constexpr int OFF_Q = 0;                     // Q0, Q1
+  static constexpr int OFF_K = 2 * TILE_BYTES;        // + s * 2 * TILE_BYTES
+  static constexpr int OFF_V = 3 * TILE_BYTES;        // + s * 2 * TILE_BYTES
+  static constexpr int OFF_BAR = TILE_BYTES * (2 + 2 * STAGES);
+  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
+  static constexpr int NUM_BARS = 1 + 2 * STAGES + 7;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;  // tmem slot, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
-  // ask for more than half an SM's shared memory so one CTA owns the TMEM
-  static constexpr int SMEM_ALLOC = (SMEM_BYTES + 1024 > 120 * 1024) ? SMEM_BYTES + 1024 : 120 * 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;     // slack for 1024-byte alignment
+  static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256, COL_P = 384;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 of the largest P entry
 };
 
 struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   int N;
-  int H;
-  int n_qtiles;
+  int n_qtiles;  // ceil(N / 128)
+  int n_pairs;   // ceil(n_qtiles / 2)
   int causal;
   float scale_log2;  // scale * log2(e)
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte alignment for the swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qtile = p.n_qtiles - 1 - static_cast<int>(blockIdx.x);  // heaviest causal tiles first
+  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x);  // heaviest causal pairs first
   const int bh = blockIdx.y;
-  const int q0 = qtile * C::BM;
   const int n_kv_total = (p.N + C::BN - 1) / C::BN;
-  const int n_kv = p.causal ? min(n_kv_total, qtile + 1) : n_kv_total;
+  // query tiles 2*pair and 2*pair+1; with causal masking tile t sees key tiles [0, qt_t]
+  const int qt0 = 2 * pair;
+  const int qt1 = 2 * pair + 1;
+  const int n0 = p.causal ? min(n_kv_total, qt0 + 1) : n_kv_total;
+  const int n1 = p.causal ? min(n_kv_total, qt1 + 1) : n_kv_total;  // n1 >= n0
+#ifdef FA2_TRACE
+  const bool trace_cta = blockIdx.x == 0 && blockIdx.y == 7;
+#endif
 
   const uint32_t bar_q = sbase + C::OFF_BAR;
   auto bar_kv_full = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + s); };
   auto bar_kv_empty = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + C::STAGES + s); };
-  auto bar_s_full = [&](int b) { return sbase + C::OFF_BAR + 8 * (1 + 2 * C::STAGES + b); };
-  const uint32_t bar_p_full = sbase + C::OFF_BAR + 8 * (3 + 2 * C::STAGES);
-  const uint32_t bar_o_done = sbase + C::OFF_BAR + 8 * (4 + 2 * C::STAGES);
-  const uint32_t bar_drain = sbase + C::OFF_BAR + 8 * (5 + 2 * C::STAGES);
+  const uint32_t bar_base = sbase + C::OFF_BAR + 8 * (1 + 2 * C::STAGES);
+  auto bar_s_full = [&](int t) { return bar_base + 8 * t; };
+  auto bar_p_full = [&](int t) { return bar_base + 16 + 8 * t; };
+  auto bar_o_done = [&](int t) { return bar_base + 32 + 8 * t; };
+  const uint32_t bar_drain = bar_base + 48;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -96,19 +112,20 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar_kv_full(s), 1);
       mbar_init(bar_kv_empty(s), 1);
     }
-    mbar_init(bar_s_full(0), 1);
-    mbar_init(bar_s_full(1), 1);
-    mbar_init(bar_p_full, 128);
-    mbar_init(bar_o_done, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full(t), 1);
+      mbar_init(bar_p_full(t), 128);
+      mbar_init(bar_o_done(t), 1);
+    }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
@@ -118,16 +135,19 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, C::TILE_BYTES);
-      for (int c = 0; c < C::CHUNKS; ++c)
-        tma_load_3d(sbase + C::OFF_Q + c * C::CHUNK_BYTES, &tm_q, bar_q, c * 64, q0, bh);
+      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+      for (int c = 0; c < C::CHUNKS; ++c) {
+        tma_load_3d(sbase + C::OFF_Q + c * C::CHUNK_BYTES, &tm_q, bar_q, c * 64, qt0 * C::BM, bh);
+        tma_load_3d(sbase + C::OFF_Q + C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar_q, c * 64,
+                    qt1 * C::BM, bh);
+      }
       int last_parity[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) last_parity[s] = -1;
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
+      for (int j = 0; j < n1 && ok; ++j) {
         const int s = j % C::STAGES;
         const int n = j / C::STAGES;
         if (n > 0) ok = mbar_wait(bar_kv_empty(s), (n - 1) & 1, abort_flag, 0x101);
@@ -146,135 +166,205 @@ __global__ void __launch_bounds__(192, 1)
       for (int s = 0; s < C::STAGES; ++s)
         if (last_parity[s] >= 0) mbar_wait(bar_kv_full(s), last_parity[s], abort_flag, 0x103);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // --------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(128, C::BN, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
-      bool ok = mbar_wait(bar_q, 0, abort_flag, 0x201);
-      auto issue_pv = [&](int t) -> bool {
-        if (!mbar_wait(bar_p_full, t & 1, abort_flag, 0x202)) return false;
-        tc_fence_after();
-        const uint32_t vbase = sbase + C::OFF_V + (t % C::STAGES) * 2 * C::TILE_BYTES;
-#pragma unroll
-        for (int k = 0; k < C::BN / 16; ++k) {
-          // V: MN-major (d contiguous), 16 keys = 2 swizzle atoms of 8 rows
-          const uint64_t bdesc = sdesc_sw128(vbase + k * 16 * 128, C::CHUNK_BYTES, 1024);
-          umma_ts(tmem + C::COL_O, tmem + C::COL_P + k * 8, bdesc, IDESC_O, (t > 0 || k > 0) ? 1u : 0u);
-        }
-        umma_commit(bar_o_done);
-        umma_commit(bar_kv_empty(t % C::STAGES));
-        return true;
-      };
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int s = j % C::STAGES;
-        const int b = j & 1;
-        ok = mbar_wait(bar_kv_full(s), (j / C::STAGES) & 1, abort_flag, 0x203);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kbase = sbase + C::OFF_K + s * 2 * C::TILE_BYTES;
+      auto issue_s = [&](int t, int j) {
+        const uint32_t kbase = sbase + C::OFF_K + (j % C::STAGES) * 2 * C::TILE_BYTES;
+        const uint32_t qbase = sbase + C::OFF_Q + t * C::TILE_BYTES;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
-          const uint64_t adesc = sdesc_sw128(sbase + C::OFF_Q + off, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(kbase + off, 16, 1024);
-          umma_ss(tmem + (b ? C::COL_S1 : C::COL_S0), adesc, bdesc, IDESC_S, k > 0 ? 1u : 0u);
+          umma_ss(tmem + (t ? C::COL_S1 : C::COL_S0), sdesc_sw128(qbase + off, 16, 1024),
+                  sdesc_sw128(kbase + off, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
         }
-        umma_commit(bar_s_full(b));
-        if (j > 0) ok = issue_pv(j - 1);
+        umma_commit(bar_s_full(t));
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t vbase = sbase + C::OFF_V + (j % C::STAGES) * 2 * C::TILE_BYTES;
+        const uint32_t pcol = tmem + (t ? C::COL_S1 : C::COL_S0);
+        const uint32_t ocol = tmem + (t ? C::COL_O1 : C::COL_O0);
+#pragma unroll
+        for (int k = 0; k < C::BN / 16; ++k) {
+          // V: MN-major (d contiguous), 16 keys = 2 swizzle atoms of 8 rows
+          umma_ts(ocol, pcol + k * 8, sdesc_sw128(vbase + k * 16 * 128, C::CHUNK_BYTES, 1024),
+                  IDESC_O, (j > 0 || k > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar_q, 0, abort_flag, 0x201) &&
+                mbar_wait(bar_kv_full(0), 0, abort_flag, 0x202);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
-      if (ok && n_kv > 0) issue_pv(n_kv - 1);
+      int kv_waited = 0;  // highest key tile whose kv_full has been waited for
+      auto wait_kv = [&](int j) -> bool {
+        if (j <= kv_waited) return true;
+        kv_waited = j;
+        if (!mbar_wait(bar_kv_full(j % C::STAGES), (j / C::STAGES) & 1, abort_flag, 0x203)) return false;
+        tc_fence_after();
+        return true;
+      };
+      for (int j = 0; j < n1 && ok; ++j) {
+        if (j < n0) {
+          ok = mbar_wait(bar_p_full(0), j & 1, abort_flag, 0x204);
+          if (!ok) break;
+          FA2_TRACE_AT(trace_cta, 16, j);
+          tc_fence_after();
+          issue_pv(0, j);
+          if (j + 1 < n0) {
+            ok = wait_kv(j + 1);
+            if (!ok) break;
+            issue_s(0, j + 1);  // overwrites S0/P0 after PV0_j in issue order
+            FA2_TRACE_AT(trace_cta, 17, j);
+          } else {
+            umma_commit(bar_o_done(0));
+          }
+        }
+        ok = mbar_wait(bar_p_full(1), j & 1, abort_flag, 0x205);
+        if (!ok) break;
+        FA2_TRACE_AT(trace_cta, 18, j);
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(bar_kv_empty(j % C::STAGES));  // K_j and V_j fully consumed
+        if (j + 1 < n1) {
+          ok = wait_kv(j + 1);
+          if (!ok) break;
+          issue_s(1, j + 1);
+          FA2_TRACE_AT(trace_cta, 19, j);
+        } else {
+          umma_commit(bar_o_done(1));
+        }
+      }
       // drain: every UMMA of this CTA has finished before TMEM is released
       umma_commit(bar_drain);
-      mbar_wait(bar_drain, 0, abort_flag, 0x401);
+      mbar_wait(bar_drain, 0, abort_flag, 0x206);
     }
   } else {
     // ---------------------------------------------------------- softmax warps
-    const int row = threadIdx.x;  // 0..127 == TMEM lane
-    const int qrow = q0 + row;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int t = warp >> 2;              // query tile of this warpgroup
+    const int row = threadIdx.x & 127;    // TMEM lane
+    const int qt = t ? qt1 : qt0;
+    const int n_t = t ? n1 : n0;
+    const int qrow = qt * C::BM + row;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t scol = t ? C::COL_S1 : C::COL_S0;
+    const uint32_t ocol = t ? C::COL_O1 : C::COL_O0;
     const float c = p.scale_log2;
-    float m = -INFINITY;  // running max of c * s, base-2 units
-    float l = 0.f;
+    float m = -INFINITY;  // reference max of c * s, base-2 units
+    float l = 0.f;        // row sum of the weights 2^(c s - m)
+    float lr = 0.f;       // the same sum over the weights rounded to bf16
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int b = j & 1;
-      ok = mbar_wait(bar_s_full(b), (j >> 1) & 1, abort_flag, 0x301);
+#ifdef FA2_TRACE
+    const bool trace_row = trace_cta && row == 0;
+#endif
+    for (int j = 0; j < n_t; ++j) {
+      FA2_TRACE_AT(trace_row, 8 * t + 0, j);
+      ok = mbar_wait(bar_s_full(t), j & 1, abort_flag, 0x301);
       if (!ok) break;
+      FA2_TRACE_AT(trace_row, 8 * t + 1, j);
       tc_fence_after();
-      const uint32_t scol = b ? C::COL_S1 : C::COL_S0;
-      float s[128];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + scol + 32 * q, *reinterpret_cast<float(*)[32]>(&s[32 * q]));
+      // pass 1: row max over the 128 scores, read from TMEM in two halves
       const int k0 = j * C::BN;
-      const bool need_mask = (p.causal && j == qtile) || (k0 + C::BN > p.N);
-      if (need_mask) {
-        const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys [0, lim) allowed
+      const bool need_mask = (p.causal && j == qt) || (k0 + C::BN > p.N);
+      const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys [0, lim) allowed
+      float mx = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (k0 + i >= lim) s[i] = -INFINITY;
-      }
-      float mx = s[0];
+      for (int h = 0; h < 2; ++h) {
+        float s[64];
+        tmem_ld64(lane_base + scol + 64 * h, s);
+        if (need_mask) {
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
-      const float m_new = fmaxf(m, mx * c);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2(m - m_use);
-      float rs = 0.f;
-      uint32_t pk[64];
-      if (!need_mask) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2(fmaf(s[2 * i], c, -m_use));
-          const float p1 = ex2(fmaf(s[2 * i + 1], c, -m_use));
-          rs += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
+          for (int i = 0; i < 64; ++i)
+            if (k0 + 64 * h + i >= lim) s[i] = -INFINITY;
         }
-      } else {
-        // masked keys contribute exactly 0 (also when c == 0, where -inf * c is NaN)
+        float a = s[0], b = s[1];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = s[2 * i] == -INFINITY ? 0.f : ex2(fmaf(s[2 * i], c, -m_use));
-          const float p1 = s[2 * i + 1] == -INFINITY ? 0.f : ex2(fmaf(s[2 * i + 1], c, -m_use));
-          rs += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
+        for (int i = 2; i < 64; i += 4) {
+          a = max3(a, s[i], s[i + 1]);
+          b = max3(b, s[i + 2], s[i + 3]);
         }
+        mx = max3(mx, a, b);
       }
-      l = l * alpha + rs;
-      m = m_use;
-      if (j > 0) {
-        // PV_{j-1} must be done before O is rescaled and before P is overwritten
-        ok = mbar_wait(bar_o_done, (j - 1) & 1, abort_flag, 0x302);
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-          for (int q = 0; q < D / 32; ++q) {
-            float o[32];
-            tmem_ld32(lane_base + C::COL_O + 32 * q, o);
-            uint32_t u[32];
+      FA2_TRACE_AT(trace_row, 8 * t + 2, j);
+      const float m_cand = fmaxf(m, mx * c);
+      const bool grow = m_cand - m > C::RESCALE_THRESHOLD;  // always true for the first tile
+      const float alpha = grow ? ex2(m - m_cand) : 1.f;
+      if (grow) m = m_cand;
+      // pass 2: weights 2^(c s - m) in pairs, written back over S as bf16 P.
+      // rs: sum of the fp32 weights (for LSE); rr: sum of the bf16-rounded weights
+      // that the P V product actually uses (for O / l, so O stays a convex
+      // combination of V rows even when one weight dominates)
+      const unsigned long long c2 = f2(c, c), negm2 = f2(-m, -m);
+      unsigned long long rs2 = f2(0.f, 0.f), rr2 = f2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(o[i] * alpha);
-            tmem_st32(lane_base + C::COL_O + 32 * q, u);
+      for (int h = 0; h < 2; ++h) {
+        float s[64];
+        tmem_ld64(lane_base + scol + 64 * h, s);
+        uint32_t pk[32];
+        if (!need_mask) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float x0, x1;
+            f2_split(f2_fma(f2(s[2 * i], s[2 * i + 1]), c2, negm2), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            const uint32_t w = pack_bf16(p0, p1);
+            pk[i] = w;
+            rs2 = f2_add(rs2, f2(p0, p1));
+            rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+          }
+        } else {
+          // masked keys contribute exactly 0 (also when c == 0, where -inf * c is NaN)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int kk = k0 + 64 * h + 2 * i;
+            const float p0 = kk >= lim ? 0.f : ex2(fmaf(s[2 * i], c, -m));
+            const float p1 = kk + 1 >= lim ? 0.f : ex2(fmaf(s[2 * i + 1], c, -m));
+            const uint32_t w = pack_bf16(p0, p1);
+            pk[i] = w;
+            rs2 = f2_add(rs2, f2(p0, p1));
+            rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
           }
         }
+        // P for keys [64h, 64h+64) goes to columns [32h, 32h+32): S there is already consumed
+        tmem_st32(lane_base + scol + 32 * h, pk);
       }
-      tmem_st32(lane_base + C::COL_P, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(lane_base + C::COL_P + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      FA2_TRACE_AT(trace_row, 8 * t + 3, j);
+      float rs_lo, rs_hi, rr_lo, rr_hi;
+      f2_split(rs2, rs_lo, rs_hi);
+      f2_split(rr2, rr_lo, rr_hi);
+      l = l * alpha + (rs_lo + rs_hi);
+      lr = lr * alpha + (rr_lo + rr_hi);
+      // O holds PV_0..PV_{j-1}: all complete, since S_j was issued after them
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+        for (int q = 0; q < D / 32; ++q) {
+          float o[32];
+          tmem_ld32(lane_base + ocol + 32 * q, o);
+          uint32_t u[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(o[i] * alpha);
+          tmem_st32(lane_base + ocol + 32 * q, u);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p_full);
+      mbar_arrive(bar_p_full(t));
+      FA2_TRACE_AT(trace_row, 8 * t + 4, j);
     }
-    if (ok && n_kv > 0) ok = mbar_wait(bar_o_done, (n_kv - 1) & 1, abort_flag, 0x303);
+    if (ok && n_t > 0) ok = mbar_wait(bar_o_done(t), 0, abort_flag, 0x303);
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / lr;
       const bool store = qrow < p.N;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + qrow) * D;
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
         float o[32];
-        tmem_ld32(lane_base + C::COL_O + 32 * q, o);
+        tmem_ld32(lane_base + ocol + 32 * q, o);
         uint4 w[4];
         uint32_t* wu = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
@@ -293,7 +383,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fa2
