@@ -15,13 +15,8 @@
 //      multiple of 128: D = 0, LSE = +inf there so P vanishes), dQ accumulator
 //      zeroed. HBM-bound.
 //   2. fa2_bwd_kernel: one CTA per (128-key block, batch*head), parallel over key
-//      blocks. K_j, V_j stay in shared memory; query blocks i stream through a
-//      TMA ring (causal: only i >= j). Per block: S^T = K Q_i^T and dP^T = V dO_i^T
-//      into tensor memory (keys on TMEM lanes), four warps (one key row per
-//      thread) form P^T and dS^T in bf16 into swizzled shared memory; then
-//      dV += P^T dO_i, dK += dS^T Q_i (accumulated in TMEM across all i) and
-//      dQ_i = dS K_j (the same dS^T buffer read MN-major), which the four warps
-//      add into the fp32 accumulator with vector reductions.
+//      blocks; dK and dV accumulate in tensor memory over all query blocks, dQ
+//      is added into an fp32 accumulator with reductions (layout below).
 //   3. fa2_bwd_dq_convert: dQ = bf16(scale * accumulator).
 #pragma once
 
@@ -114,36 +109,60 @@ __global__ void __launch_bounds__(256) fa2_bwd_dq_convert_kernel(const BwdConver
   }
 }
 
+
 // ------------------------------------------------------------ main kernel (B2)
+// One CTA per (128-key block j, batch*head); query blocks i stream through a
+// two-stage TMA ring (causal: only i >= j, the diagonal block first).
+//   warp 8        TMA producer: K_j, V_j once; Q_i, dO_i, LSE2_i, D_i per step
+//   warp 9        MMA issuer + TMEM owner, per step:
+//                   S^T = K Q_i^T,  dP^T = V dO_i^T          (keys on TMEM lanes)
+//                   dV += P^T dO_i    (P^T from TMEM)
+//                   dK += dS^T Q_i    (dS^T from smem, K-major)
+//                   d = 128: dQ^T = K^T dS^T (d on lanes; dS^T read MN-major)
+//                   d =  64: dQ   = dS K     (queries on lanes)
+//   warps 0-3     query columns [0, 64) of the step, warps 4-7 columns [64, 128):
+//                 thread r owns key row r. P^T = exp2(c S^T - LSE2) goes back
+//                 into TMEM over the half's own S^T columns; dS^T = P^T (dP^T - D)
+//                 goes to swizzled smem; then the half drains its share of dQ
+//                 into the fp32 accumulator with reductions.
+// Tensor memory: S^T [0,128) (P^T in [0,32) and [64,96)), dP^T [128,256),
+// dV [256,256+D), dK [256+D,256+2D); dQ^T (d = 128) reuses the dP^T columns once
+// dS is in smem, dQ (d = 64) has [384,448).
 template <int D>
 struct BwdCfg {
   static_assert(D == 64 || D == 128, "head dim");
   static constexpr int BM = 128;                      // query rows per step
   static constexpr int BN = 128;                      // keys per CTA
-  static constexpr int STAGES = (D == 64) ? 2 : 1;
+  static constexpr int STAGES = 2;
   static constexpr int CHUNKS = D / 64;
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int CHUNK_BYTES = 128 * 128;
   static constexpr int VEC_BYTES = 512;               // 128 fp32
-  // Q, dO, LSE2, D (+ padding to keep the next stage's tiles 1024-byte aligned)
-  static constexpr int STAGE_STRIDE = 2 * TILE_BYTES + 1024;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = TILE_BYTES;
-  static constexpr int OFF_ST = 2 * TILE_BYTES;                              // + s * STAGE_STRIDE
-  static constexpr int ST_Q = 0, ST_DO = TILE_BYTES, ST_LSE = 2 * TILE_BYTES, ST_D = 2 * TILE_BYTES + VEC_BYTES;
-  static constexpr int OFF_PT = OFF_ST + STAGES * STAGE_STRIDE;             // 128 x 128 bf16
-  static constexpr int OFF_DST = OFF_PT + 32768;
-  static constexpr int OFF_BAR = OFF_DST + 32768;
-  // kv_full, st_full[S], st_empty[S], s_full, dp_full, ds_ready, pds_free,
-  // dq_full, dq_empty, dkv_done, drain
-  static constexpr int NUM_BARS = 1 + 2 * STAGES + 8;
+  static constexpr int OFF_Q = 2 * TILE_BYTES;                    // + s * TILE_BYTES
+  static constexpr int OFF_DO = OFF_Q + STAGES * TILE_BYTES;      // + s * TILE_BYTES
+  static constexpr int OFF_DS = OFF_DO + STAGES * TILE_BYTES;     // 128 x 128 bf16
+  static constexpr int OFF_VEC = OFF_DS + 32768;                  // [s][LSE2 | D]
+  static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
+  // kv_full, st_full[S], st_empty[S], s_full, dp_full, p_ready, ds_ready,
+  // dsm_free, dq_full, dq_empty, dkv_done, drain
+  static constexpr int NUM_BARS = 1 + 2 * STAGES + 9;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
-  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-  static constexpr int THREADS = 192;
+  // d = 128 uses 231,6xx bytes: there is no room for alignment slack, so the
+  // kernel checks that the dynamic shared memory base is 1024-byte aligned
+  static constexpr bool NEEDS_ALIGNED_BASE = SMEM_BYTES + 1024 > 232448;
+  static constexpr int SMEM_ALLOC = NEEDS_ALIGNED_BASE ? SMEM_BYTES : SMEM_BYTES + 1024;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-  // d = 128 has no room left: dQ reuses the dP^T columns once dS is in smem
+  // dQ layout: d = 128 computes dQ^T (d on lanes), so each warp reduction adds
+  // 128 contiguous bytes of one query row: measured faster than 16-byte vector
+  // reductions over scattered rows, which the L2 handles per half-filled sector.
+  // d = 64 cannot (M would be 64) and uses dQ with queries on lanes.
+  static constexpr bool DQ_T = (D == 128);
+  // d = 128 has no free columns left: dQ reuses the dP^T columns once dS is in smem
   static constexpr bool DQ_IN_DP = (D == 128);
   static constexpr uint32_t COL_DQ = DQ_IN_DP ? COL_DP : 256 + 2 * D;
 };
@@ -168,6 +187,10 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+__device__ __forceinline__ void red_add(float* addr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
+}
+
 // Byte offset of 16-byte unit u (0..15) of row r in a [128][128] bf16 tile
 // stored as two K-major 128-byte-swizzled halves of 64 columns.
 __device__ __forceinline__ uint32_t sw128_offset(int r, int u) {
@@ -175,35 +198,46 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int u) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (C::NEEDS_ALIGNED_BASE && (smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_timeout(0x1000);  // layout assumption broken: refuse to run
+    return;
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ktile = blockIdx.x;  // causal: low key blocks see the most query blocks; run them first
+  // grid (key tile, batch*head): the key blocks of one head run together and
+  // share its Q/dO tiles in L2 (measured faster than a longest-first order
+  // across heads, even for causal masks)
+  const int ktile = blockIdx.x;
   const int bh = blockIdx.y;
   const int k0 = ktile * C::BN;
   const int n_qtiles = p.n_ktiles;  // self-attention: same N
   const int i_first = p.causal ? ktile : 0;
   const int n_iter = n_qtiles - i_first;
+#ifdef FA2_TRACE
+  const bool trace_cta = blockIdx.x == 0 && blockIdx.y == 7;
+#endif
 
   const uint32_t bar_kv = sbase + C::OFF_BAR;
   auto bar_st_full = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + s); };
   auto bar_st_empty = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + C::STAGES + s); };
   const uint32_t bar_s_full = sbase + C::OFF_BAR + 8 * (1 + 2 * C::STAGES);
   const uint32_t bar_dp_full = bar_s_full + 8;
-  const uint32_t bar_ds_ready = bar_s_full + 16;
-  const uint32_t bar_pds_free = bar_s_full + 24;
-  const uint32_t bar_dq_full = bar_s_full + 32;
-  const uint32_t bar_dq_empty = bar_s_full + 40;
-  const uint32_t bar_dkv_done = bar_s_full + 48;
-  const uint32_t bar_drain = bar_s_full + 56;
+  const uint32_t bar_p_ready = bar_s_full + 16;
+  const uint32_t bar_ds_ready = bar_s_full + 24;
+  const uint32_t bar_dsm_free = bar_s_full + 32;
+  const uint32_t bar_dq_full = bar_s_full + 40;
+  const uint32_t bar_dq_empty = bar_s_full + 48;
+  const uint32_t bar_dkv_done = bar_s_full + 56;
+  const uint32_t bar_drain = bar_s_full + 64;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -215,20 +249,21 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
-    mbar_init(bar_ds_ready, 128);
-    mbar_init(bar_pds_free, 1);
+    mbar_init(bar_p_ready, 256);
+    mbar_init(bar_ds_ready, 256);
+    mbar_init(bar_dsm_free, 1);
     mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_empty, 128);
+    mbar_init(bar_dq_empty, 256);
     mbar_init(bar_dkv_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
@@ -239,7 +274,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
@@ -256,193 +291,274 @@ __global__ void __launch_bounds__(192, 1)
         const int n = it / C::STAGES;
         if (n > 0) ok = mbar_wait(bar_st_empty(s), (n - 1) & 1, abort_flag, 0x1101);
         if (!ok) break;
-        const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_STRIDE;
         const uint32_t bar = bar_st_full(s);
         mbar_arrive_expect_tx(bar, 2 * C::TILE_BYTES + 2 * C::VEC_BYTES);
         for (int c = 0; c < C::CHUNKS; ++c) {
-          tma_load_3d(st + C::ST_Q + c * C::CHUNK_BYTES, &tm_q, bar, c * 64, i * C::BM, bh);
-          tma_load_3d(st + C::ST_DO + c * C::CHUNK_BYTES, &tm_do, bar, c * 64, i * C::BM, bh);
+          tma_load_3d(sbase + C::OFF_Q + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar, c * 64,
+                      i * C::BM, bh);
+          tma_load_3d(sbase + C::OFF_DO + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do, bar,
+                      c * 64, i * C::BM, bh);
         }
         const size_t voff = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * C::BM;
-        bulk_load(st + C::ST_LSE, p.lse2 + voff, C::VEC_BYTES, bar);
-        bulk_load(st + C::ST_D, p.delta + voff, C::VEC_BYTES, bar);
+        const uint32_t vec = sbase + C::OFF_VEC + s * 2 * C::VEC_BYTES;
+        bulk_load(vec, p.lse2 + voff, C::VEC_BYTES, bar);
+        bulk_load(vec + C::VEC_BYTES, p.delta + voff, C::VEC_BYTES, bar);
         last_parity[s] = n & 1;
       }
       mbar_wait(bar_kv, 0, abort_flag, 0x1102);
       for (int s = 0; s < C::STAGES; ++s)
         if (last_parity[s] >= 0) mbar_wait(bar_st_full(s), last_parity[s], abort_flag, 0x1103);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // --------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_SS = idesc_bf16(128, 128, false, false);   // S^T, dP^T
       constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);      // dV, dK
-      constexpr uint32_t IDESC_Q = idesc_bf16(128, D, true, true);        // dQ
-      bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x1201);
-      for (int it = 0; it < n_iter && ok; ++it) {
-        const int s = it % C::STAGES;
-        const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_STRIDE;
-        ok = mbar_wait(bar_st_full(s), (it / C::STAGES) & 1, abort_flag, 0x1202);
-        if (!ok) break;
-        tc_fence_after();
-        // S^T = K Q_i^T (the S columns were read before ds_ready(it-1), waited below)
+      constexpr uint32_t IDESC_QT = idesc_bf16(128, 128, true, true);     // dQ^T (d = 128)
+      constexpr uint32_t IDESC_Q = idesc_bf16(128, D, true, true);        // dQ (d = 64)
+      auto issue_s = [&](int it) {  // S^T = K Q_i^T
+        const uint32_t q_s = sbase + C::OFF_Q + (it % C::STAGES) * C::TILE_BYTES;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
           umma_ss(tmem + C::COL_S, sdesc_sw128(sbase + C::OFF_K + off, 16, 1024),
-                  sdesc_sw128(st + C::ST_Q + off, 16, 1024), IDESC_SS, k > 0 ? 1u : 0u);
+                  sdesc_sw128(q_s + off, 16, 1024), IDESC_SS, k > 0 ? 1u : 0u);
         }
         umma_commit(bar_s_full);
-        // dP^T = V dO_i^T; with d = 128 the dP columns hold dQ_{i-1} until drained
-        if (C::DQ_IN_DP && it > 0) {
+      };
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x1201) &&
+                mbar_wait(bar_st_full(0), 0, abort_flag, 0x1202);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      // Per step i: dP^T_i, dV_i, S^T_{i+1}, dK_i, dQ_i. S^T_{i+1} goes right after
+      // dV_i so that the elementwise warps can form P^T_{i+1} while the tensor
+      // core runs dK_i and dQ_i; it overwrites P^T_i only after dV_i in issue order.
+      for (int it = 0; it < n_iter && ok; ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t q_s = sbase + C::OFF_Q + s * C::TILE_BYTES;
+        const uint32_t do_s = sbase + C::OFF_DO + s * C::TILE_BYTES;
+        FA2_TRACE_AT(trace_cta, 16, it);
+        if (C::DQ_IN_DP && it > 0) {  // the dP^T columns hold dQ_{i-1} until it is read out
           ok = mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x1203);
           if (!ok) break;
           tc_fence_after();
         }
+        FA2_TRACE_AT(trace_cta, 17, it);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < D / 16; ++k) {  // dP^T = V dO_i^T
           const uint32_t off = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
           umma_ss(tmem + C::COL_DP, sdesc_sw128(sbase + C::OFF_V + off, 16, 1024),
-                  sdesc_sw128(st + C::ST_DO + off, 16, 1024), IDESC_SS, k > 0 ? 1u : 0u);
+                  sdesc_sw128(do_s + off, 16, 1024), IDESC_SS, k > 0 ? 1u : 0u);
         }
         umma_commit(bar_dp_full);
-        // P^T and dS^T are in shared memory; S^T and dP^T have been read
-        ok = mbar_wait(bar_ds_ready, it & 1, abort_flag, 0x1204);
+        // dV += P^T dO_i once both halves have written P^T
+        ok = mbar_wait(bar_p_ready, it & 1, abort_flag, 0x1204);
         if (!ok) break;
+        FA2_TRACE_AT(trace_cta, 18, it);
         tc_fence_after();
-        const uint32_t pt = sbase + C::OFF_PT;
-        const uint32_t dst = sbase + C::OFF_DST;
 #pragma unroll
         for (int k = 0; k < C::BM / 16; ++k) {
-          const uint32_t aoff = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;   // K-major over queries
-          const uint64_t bdo = sdesc_sw128(st + C::ST_DO + k * 2048, C::CHUNK_BYTES, 1024);
-          umma_ss(tmem + C::COL_DV, sdesc_sw128(pt + aoff, 16, 1024), bdo, IDESC_KV,
+          // queries 16k..16k+15: columns 8k (first half) or 64 + 8(k-4) (second half)
+          const uint32_t pcol = C::COL_S + (k < 4 ? 8 * k : 64 + 8 * (k - 4));
+          umma_ts(tmem + C::COL_DV, tmem + pcol,
+                  sdesc_sw128(do_s + k * 2048, C::CHUNK_BYTES, 1024), IDESC_KV,
                   (it > 0 || k > 0) ? 1u : 0u);
         }
+        if (it + 1 < n_iter) {
+          ok = mbar_wait(bar_st_full((it + 1) % C::STAGES), ((it + 1) / C::STAGES) & 1, abort_flag,
+                         0x1208);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(it + 1);
+        }
+        // dK += dS^T Q_i and dQ once dS^T is in smem
+        ok = mbar_wait(bar_ds_ready, it & 1, abort_flag, 0x1205);
+        if (!ok) break;
+        FA2_TRACE_AT(trace_cta, 19, it);
+        tc_fence_after();
+        const uint32_t ds = sbase + C::OFF_DS;
 #pragma unroll
         for (int k = 0; k < C::BM / 16; ++k) {
           const uint32_t aoff = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
-          const uint64_t bq = sdesc_sw128(st + C::ST_Q + k * 2048, C::CHUNK_BYTES, 1024);
-          umma_ss(tmem + C::COL_DK, sdesc_sw128(dst + aoff, 16, 1024), bq, IDESC_KV,
+          umma_ss(tmem + C::COL_DK, sdesc_sw128(ds + aoff, 16, 1024),
+                  sdesc_sw128(q_s + k * 2048, C::CHUNK_BYTES, 1024), IDESC_KV,
                   (it > 0 || k > 0) ? 1u : 0u);
         }
-        if (!C::DQ_IN_DP && it > 0) {
-          ok = mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x1205);
+        if (!C::DQ_IN_DP && it > 0) {  // dQ_{i-1} must be read out before it is overwritten
+          ok = mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x1206);
           if (!ok) break;
           tc_fence_after();
         }
-        // dQ_i = dS K_j: A = dS (queries x keys), the dS^T buffer read MN-major
 #pragma unroll
-        for (int k = 0; k < C::BN / 16; ++k) {
-          const uint64_t a = sdesc_sw128(dst + k * 2048, C::CHUNK_BYTES, 1024);
-          const uint64_t b = sdesc_sw128(sbase + C::OFF_K + k * 2048, C::CHUNK_BYTES, 1024);
-          umma_ss(tmem + C::COL_DQ, a, b, IDESC_Q, k > 0 ? 1u : 0u);
+        for (int k = 0; k < C::BN / 16; ++k) {  // reduction over the 128 keys
+          const uint64_t kdesc = sdesc_sw128(sbase + C::OFF_K + k * 2048, C::CHUNK_BYTES, 1024);
+          const uint64_t sdesc = sdesc_sw128(ds + k * 2048, C::CHUNK_BYTES, 1024);
+          if (C::DQ_T)
+            umma_ss(tmem + C::COL_DQ, kdesc, sdesc, IDESC_QT, k > 0 ? 1u : 0u);  // K^T dS^T
+          else
+            umma_ss(tmem + C::COL_DQ, sdesc, kdesc, IDESC_Q, k > 0 ? 1u : 0u);   // dS K
         }
         umma_commit(bar_dq_full);
-        umma_commit(bar_pds_free);
+        umma_commit(bar_dsm_free);
         umma_commit(bar_st_empty(s));
       }
       umma_commit(bar_dkv_done);
       umma_commit(bar_drain);
-      mbar_wait(bar_drain, 0, abort_flag, 0x1206);
+      mbar_wait(bar_drain, 0, abort_flag, 0x1207);
     }
   } else {
-    // ------------------------------------------------- P / dS / dQ warps (0-3)
-    const int r = threadIdx.x;  // key row of this CTA == TMEM lane (S^T, dP^T, dK, dV)
+    // --------------------------------------------- elementwise halves (0-3, 4-7)
+    const int h = warp >> 2;            // query-column half of this warpgroup
+    const int r = threadIdx.x & 127;    // TMEM lane: key row (S^T, dP^T, dK, dV)
     const int key = k0 + r;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.scale_log2;
-    uint8_t* pt_row = smem + C::OFF_PT;
-    uint8_t* ds_row = smem + C::OFF_DST;
+    uint8_t* ds_base = smem + C::OFF_DS;
+#ifdef FA2_TRACE
+    const bool trace_row = trace_cta && r == 0;
+#endif
+    // dQ of step it (this half's share) -> fp32 accumulator. The TMEM columns are
+    // released as soon as the values are in registers; the reductions follow.
+    auto drain = [&](int it) -> bool {
+      if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x1304)) return false;
+      FA2_TRACE_AT(trace_row, 8 * h + 4, it);
+      tc_fence_after();
+      float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i_first + it) * C::BM) * D;
+      if (C::DQ_T) {
+        // lane r holds dQ^T[d = r][query 64h + q]: each warp instruction adds 32
+        // consecutive d values of one query row (128 contiguous bytes)
+        float v[64];
+        tmem_ld64(lane_base + C::COL_DQ + 64 * h, v);
+        tc_fence_before();
+        mbar_arrive(bar_dq_empty);
+        float* col = acc + static_cast<size_t>(64 * h) * D + r;
+#pragma unroll
+        for (int q = 0; q < 64; ++q) red_add(col + static_cast<size_t>(q) * D, v[q]);
+      } else {
+        // lane r holds dQ[query r][d]; this half adds d columns [h D/2, (h+1) D/2)
+        float v[D / 2];
+        if constexpr (D == 128)
+          tmem_ld64(lane_base + C::COL_DQ + (D / 2) * h, v);
+        else
+          tmem_ld32(lane_base + C::COL_DQ + (D / 2) * h, v);
+        tc_fence_before();
+        mbar_arrive(bar_dq_empty);
+        float* row = acc + static_cast<size_t>(r) * D + (D / 2) * h;
+#pragma unroll
+        for (int e = 0; e < D / 2; e += 4) red_add_v4(row + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
+      }
+      FA2_TRACE_AT(trace_row, 8 * h + 5, it);
+      return true;
+    };
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int i = i_first + it;
       const int s = it % C::STAGES;
-      const uint8_t* st = smem + C::OFF_ST + s * C::STAGE_STRIDE;
-      const float* lse2 = reinterpret_cast<const float*>(st + C::ST_LSE);
-      const float* dlt = reinterpret_cast<const float*>(st + C::ST_D);
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 2 * C::VEC_BYTES) + 64 * h;
+      const float* dlt = lse2 + 128;
+      FA2_TRACE_AT(trace_row, 8 * h + 0, it);
       // LSE2 and D of this query block were written by the TMA (async proxy)
       ok = mbar_wait(bar_st_full(s), (it / C::STAGES) & 1, abort_flag, 0x1300);
       if (!ok) break;
       ok = mbar_wait(bar_s_full, it & 1, abort_flag, 0x1301);
       if (!ok) break;
-      ok = mbar_wait(bar_dp_full, it & 1, abort_flag, 0x1302);
-      if (!ok) break;
-      // the previous step's MMAs have finished reading P^T and dS^T
+      FA2_TRACE_AT(trace_row, 8 * h + 1, it);
+      tc_fence_after();
+      // P^T for query columns [64h, 64h + 64)
+      uint32_t pk[32];
+      {
+        float sv[64];
+        tmem_ld64(lane_base + C::COL_S + 64 * h, sv);
+        const unsigned long long c2 = f2(c, c);
+        const bool diag = p.causal && (i == ktile);
+#pragma unroll
+        for (int e = 0; e < 64; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + e);
+          float x0, x1, x2, x3;
+          f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
+          f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
+          float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+          if (diag) {  // query i*128 + q sees key k0 + r only if q >= r
+            const int q = 64 * h + e;
+            if (q < r) p0 = 0.f;
+            if (q + 1 < r) p1 = 0.f;
+            if (q + 2 < r) p2 = 0.f;
+            if (q + 3 < r) p3 = 0.f;
+          }
+          pk[e / 2] = pack_bf16(p0, p1);
+          pk[e / 2 + 1] = pack_bf16(p2, p3);
+        }
+      }
+      // P^T over this half's own first 32 S^T columns (already read above)
+      tmem_st32(lane_base + C::COL_S + 64 * h, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p_ready);
+      FA2_TRACE_AT(trace_row, 8 * h + 2, it);
+      // the previous step's dQ is ready by now (its MMAs ran while P^T was formed)
       if (it > 0) {
-        ok = mbar_wait(bar_pds_free, (it - 1) & 1, abort_flag, 0x1303);
+        ok = drain(it - 1);
         if (!ok) break;
       }
+      // dS^T = P^T (dP^T - D) for the same columns, bf16 into the swizzled smem tile
+      ok = mbar_wait(bar_dp_full, it & 1, abort_flag, 0x1302);
+      if (!ok) break;
       tc_fence_after();
-      const bool diag = p.causal && (i == ktile);
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {  // 32 query columns at a time
-        float sv[32], dp[32];
-        tmem_ld32(lane_base + C::COL_S + 32 * q, sv);
-        tmem_ld32(lane_base + C::COL_DP + 32 * q, dp);
-        uint32_t pk[16], dk[16];
+      uint32_t dk[32];
+      {
+        float dp[64];
+        tmem_ld64(lane_base + C::COL_DP + 64 * h, dp);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int col = 32 * q + e;
-          float p0 = ex2(fmaf(sv[e], c, -lse2[col]));
-          float p1 = ex2(fmaf(sv[e + 1], c, -lse2[col + 1]));
-          if (diag) {  // query i*128+col may see key k0+r only if col >= r
-            if (col < r) p0 = 0.f;
-            if (col + 1 < r) p1 = 0.f;
-          }
-          const float d0 = p0 * (dp[e] - dlt[col]);
-          const float d1 = p1 * (dp[e + 1] - dlt[col + 1]);
-          pk[e / 2] = pack_bf16(p0, p1);
-          dk[e / 2] = pack_bf16(d0, d1);
+        for (int e = 0; e < 64; e += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(dlt + e);
+          const float p0 = __uint_as_float(pk[e / 2] << 16), p1 = __uint_as_float(pk[e / 2] & 0xFFFF0000u);
+          const float p2 = __uint_as_float(pk[e / 2 + 1] << 16), p3 = __uint_as_float(pk[e / 2 + 1] & 0xFFFF0000u);
+          dk[e / 2] = pack_bf16(p0 * (dp[e] - d4.x), p1 * (dp[e + 1] - d4.y));
+          dk[e / 2 + 1] = pack_bf16(p2 * (dp[e + 2] - d4.z), p3 * (dp[e + 3] - d4.w));
         }
+      }
+      if (it > 0) {  // dK_{i-1} and dQ_{i-1} have finished reading the dS^T tile
+        ok = mbar_wait(bar_dsm_free, (it - 1) & 1, abort_flag, 0x1303);
+        if (!ok) break;
+      }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t off = sw128_offset(r, 4 * q + u);
-          *reinterpret_cast<uint4*>(pt_row + off) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-          *reinterpret_cast<uint4*>(ds_row + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-        }
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t off = sw128_offset(r, 8 * h + u);
+        *reinterpret_cast<uint4*>(ds_base + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
       }
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(bar_ds_ready);
-      // dQ_i (query rows on TMEM lanes) -> fp32 accumulator
-      ok = mbar_wait(bar_dq_full, it & 1, abort_flag, 0x1304);
-      if (!ok) break;
-      tc_fence_after();
-      float* dq_row = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * C::BM + r) * D;
-#pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
-        float v[32];
-        tmem_ld32(lane_base + C::COL_DQ + 32 * q, v);
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) red_add_v4(dq_row + 32 * q + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
-      }
-      tc_fence_before();
-      mbar_arrive(bar_dq_empty);
+      FA2_TRACE_AT(trace_row, 8 * h + 3, it);
     }
+    if (ok && n_iter > 0) ok = drain(n_iter - 1);
     if (ok) ok = mbar_wait(bar_dkv_done, 0, abort_flag, 0x1305);
     if (ok) {
+      // epilogue: this half stores d columns [h D/2, (h+1) D/2) of dV and scale * dK
       tc_fence_after();
       const bool store = key < p.N;
       const size_t off = (static_cast<size_t>(bh) * p.N + key) * D;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = 0; q < D / 64; ++q) {
+        const int c0 = h * (D / 2) + 32 * q;
         float v[32];
         uint4 w[4];
         uint32_t* wu = reinterpret_cast<uint32_t*>(w);
-        tmem_ld32(lane_base + C::COL_DV + 32 * q, v);
+        tmem_ld32(lane_base + C::COL_DV + c0, v);
 #pragma unroll
         for (int e = 0; e < 16; ++e) wu[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
         if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dv + off + 32 * q);
+          uint4* dst = reinterpret_cast<uint4*>(p.dv + off + c0);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = w[e];
         }
-        tmem_ld32(lane_base + C::COL_DK + 32 * q, v);
+        tmem_ld32(lane_base + C::COL_DK + c0, v);
 #pragma unroll
         for (int e = 0; e < 16; ++e) wu[e] = pack_bf16(v[2 * e] * p.scale, v[2 * e + 1] * p.scale);
         if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dk + off + 32 * q);
+          uint4* dst = reinterpret_cast<uint4*>(p.dk + off + c0);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = w[e];
         }
@@ -453,7 +569,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fa2

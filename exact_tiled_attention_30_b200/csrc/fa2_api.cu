@@ -89,8 +89,9 @@ fa2_status check_common(int B, int H, int N, int d, float scale) {
   if (!std::isfinite(scale) || scale < 0.f) return FA2_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA2_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > 65535) return FA2_ERR_UNSUPPORTED;
-  // every tensor index must fit the 32-bit TMA coordinates and our size_t math
-  if (static_cast<long long>(N) > (1LL << 30)) return FA2_ERR_UNSUPPORTED;
+  // every tensor index must fit the 32-bit TMA coordinates and our size_t math,
+  // and the 128-row tiles a grid dimension (at most 65535)
+  if (static_cast<long long>(N) > 65535LL * 128) return FA2_ERR_UNSUPPORTED;
   return FA2_OK;
 }
 
@@ -130,7 +131,7 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   p.n_pairs = (p.n_qtiles + 1) / 2;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
-  dim3 grid(p.n_pairs, BH);
+  const dim3 grid = p.causal ? dim3(BH, p.n_pairs) : dim3(p.n_pairs, BH);
   fa2::fa2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
   return FA2_OK;

@@ -83,8 +83,12 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x);  // heaviest causal pairs first
-  const int bh = blockIdx.y;
+  // Blocks launch in linear order. Causal: grid (batch*head, pair) with the pair
+  // as the slow index, so the heaviest pairs of all heads start first (longest
+  // processing time first). Non-causal: grid (pair, batch*head), so the pairs of
+  // one head run together and share its K/V tiles in L2.
+  const int pair = p.causal ? p.n_pairs - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
+  const int bh = p.causal ? blockIdx.x : blockIdx.y;
   const int n_kv_total = (p.N + C::BN - 1) / C::BN;
   // query tiles 2*pair and 2*pair+1; with causal masking tile t sees key tiles [0, qt_t]
   const int qt0 = 2 * pair;
@@ -92,7 +96,7 @@ __global__ void __launch_bounds__(320, 1)
   const int n0 = p.causal ? min(n_kv_total, qt0 + 1) : n_kv_total;
   const int n1 = p.causal ? min(n_kv_total, qt1 + 1) : n_kv_total;  // n1 >= n0
 #ifdef FA2_TRACE
-  const bool trace_cta = blockIdx.x == 0 && blockIdx.y == 7;
+  const bool trace_cta = blockIdx.y == 0 && blockIdx.x == 7;
 #endif
 
   const uint32_t bar_q = sbase + C::OFF_BAR;

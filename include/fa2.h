@@ -24,7 +24,7 @@
  *  - Tensors q, k, v, o, dO, dq, dk, dv are bf16, contiguous [B, H, N, d]
  *    (row-major; d innermost). Q and K/V have the same length N
  *    (self-attention). lse is fp32 [B, H, N].
- *  - d must be 64 or 128. N >= 1 (any N; the last tile is masked).
+ *  - d must be 64 or 128. 1 <= N <= 65535 * 128 (any N; the last tile is masked).
  *    B >= 1, H >= 1, B * H <= 65535.
  *  - scale must be finite and >= 0 (typically 1/sqrt(d)).
  *  - All pointers are device pointers (HBM), 16-byte aligned (the kernels load
