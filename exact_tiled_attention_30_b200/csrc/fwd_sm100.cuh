@@ -34,6 +34,7 @@
 // a convex combination of V rows when one weight dominates; LSE uses the fp32 sum.
 #pragma once
 
+#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa2 {
@@ -60,6 +61,9 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
   static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 of the largest P entry
+  // d = 64: one pair of weights in POLY_EVERY is exponentiated on the FMA pipe
+  // (the MUFU unit is the tighter limit there); d = 128: MUFU only (measured faster)
+  static constexpr int POLY_EVERY = (D == 64) ? 3 : 1 << 20;
 };
 
 struct FwdParams {
@@ -312,9 +316,14 @@ __global__ void __launch_bounds__(320, 1)
         if (!need_mask) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            float x0, x1;
+            float x0, x1, p0, p1;
             f2_split(f2_fma(f2(s[2 * i], s[2 * i + 1]), c2, negm2), x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);
+            if (i % C::POLY_EVERY == C::POLY_EVERY - 1) {
+              exp2_poly2(x0, x1, p0, p1);  // FMA pipe: balances the MUFU unit
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
             const uint32_t w = pack_bf16(p0, p1);
             pk[i] = w;
             rs2 = f2_add(rs2, f2(p0, p1));
