@@ -113,19 +113,21 @@ __global__ void __launch_bounds__(256) fa2_bwd_dq_convert_kernel(const BwdConver
 // ------------------------------------------------------------ main kernel (B2)
 // One CTA per (128-key block j, batch*head); query blocks i stream through a
 // two-stage TMA ring (causal: only i >= j, the diagonal block first).
-//   warp 8        TMA producer: K_j, V_j once; Q_i, dO_i, LSE2_i, D_i per step
-//   warp 9        MMA issuer + TMEM owner, per step:
+//   warp 16       TMA producer: K_j, V_j once; Q_i, dO_i, LSE2_i, D_i per step
+//   warp 17       MMA issuer + TMEM owner, per step:
 //                   S^T = K Q_i^T,  dP^T = V dO_i^T          (keys on TMEM lanes)
 //                   dV += P^T dO_i    (P^T from TMEM)
 //                   dK += dS^T Q_i    (dS^T from smem, K-major)
 //                   d = 128: dQ^T = K^T dS^T (d on lanes; dS^T read MN-major)
 //                   d =  64: dQ   = dS K     (queries on lanes)
-//   warps 0-3     query columns [0, 64) of the step, warps 4-7 columns [64, 128):
-//                 thread r owns key row r. P^T = exp2(c S^T - LSE2) goes back
-//                 into TMEM over the half's own S^T columns; dS^T = P^T (dP^T - D)
-//                 goes to swizzled smem; then the half drains its share of dQ
-//                 into the fp32 accumulator with reductions.
-// Tensor memory: S^T [0,128) (P^T in [0,32) and [64,96)), dP^T [128,256),
+//   warps 0-15    four elementwise warpgroups; warpgroup g owns query columns
+//                 [32g, 32g + 32) of the step and thread r key row r. P^T =
+//                 exp2(c S^T - LSE2) goes back into TMEM over the group's own
+//                 S^T columns; dS^T = P^T (dP^T - D) goes to swizzled smem; then
+//                 the group adds its share of dQ into the fp32 accumulator with
+//                 reductions. No row statistics are needed (P comes from the
+//                 saved LSE), so the groups never exchange data.
+// Tensor memory: S^T [0,128) (P^T of group g in [32g, 32g+16)), dP^T [128,256),
 // dV [256,256+D), dK [256+D,256+2D); dQ^T (d = 128) reuses the dP^T columns once
 // dS is in smem, dQ (d = 64) has [384,448).
 template <int D>
@@ -154,7 +156,11 @@ struct BwdCfg {
   // kernel checks that the dynamic shared memory base is 1024-byte aligned
   static constexpr bool NEEDS_ALIGNED_BASE = SMEM_BYTES + 1024 > 232448;
   static constexpr int SMEM_ALLOC = NEEDS_ALIGNED_BASE ? SMEM_BYTES : SMEM_BYTES + 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int NWG = 4;                       // elementwise warpgroups
+  static constexpr int CW = 128 / NWG;                 // query columns per group
+  static constexpr int WARP_TMA = 4 * NWG, WARP_MMA = 4 * NWG + 1;
+  static constexpr int THREADS = 32 * (4 * NWG + 2);
+  static constexpr int ELEM_THREADS = 128 * NWG;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   // dQ layout: d = 128 computes dQ^T (d on lanes), so each warp reduction adds
@@ -198,7 +204,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int u) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const BwdParams p) {
@@ -249,21 +255,21 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
-    mbar_init(bar_p_ready, 256);
-    mbar_init(bar_ds_ready, 256);
+    mbar_init(bar_p_ready, C::ELEM_THREADS);
+    mbar_init(bar_ds_ready, C::ELEM_THREADS);
     mbar_init(bar_dsm_free, 1);
     mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_empty, 256);
+    mbar_init(bar_dq_empty, C::ELEM_THREADS);
     mbar_init(bar_dkv_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == C::WARP_TMA && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == C::WARP_TMA) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
@@ -309,7 +315,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int s = 0; s < C::STAGES; ++s)
         if (last_parity[s] >= 0) mbar_wait(bar_st_full(s), last_parity[s], abort_flag, 0x1103);
     }
-  } else if (warp == 9) {
+  } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_SS = idesc_bf16(128, 128, false, false);   // S^T, dP^T
@@ -360,8 +366,8 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < C::BM / 16; ++k) {
-          // queries 16k..16k+15: columns 8k (first half) or 64 + 8(k-4) (second half)
-          const uint32_t pcol = C::COL_S + (k < 4 ? 8 * k : 64 + 8 * (k - 4));
+          // queries 16k..16k+15 sit in group g = 16k / CW at column CW g + (16k mod CW) / 2
+          const uint32_t pcol = C::COL_S + C::CW * ((16 * k) / C::CW) + ((16 * k) % C::CW) / 2;
           umma_ts(tmem + C::COL_DV, tmem + pcol,
                   sdesc_sw128(do_s + k * 2048, C::CHUNK_BYTES, 1024), IDESC_KV,
                   (it > 0 || k > 0) ? 1u : 0u);
@@ -409,79 +415,81 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait(bar_drain, 0, abort_flag, 0x1207);
     }
   } else {
-    // --------------------------------------------- elementwise halves (0-3, 4-7)
-    const int h = warp >> 2;            // query-column half of this warpgroup
+    // ------------------------------------------------ elementwise groups (0-15)
+    constexpr int CW = C::CW;
+    const int g = warp >> 2;            // query-column group
     const int r = threadIdx.x & 127;    // TMEM lane: key row (S^T, dP^T, dK, dV)
     const int key = k0 + r;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.scale_log2;
     uint8_t* ds_base = smem + C::OFF_DS;
 #ifdef FA2_TRACE
-    const bool trace_row = trace_cta && r == 0;
+    const bool trace_row = trace_cta && r == 0 && g < 2;
 #endif
-    // dQ of step it (this half's share) -> fp32 accumulator. The TMEM columns are
+    // dQ of step it (this group's share) -> fp32 accumulator. The TMEM columns are
     // released as soon as the values are in registers; the reductions follow.
     auto drain = [&](int it) -> bool {
       if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x1304)) return false;
-      FA2_TRACE_AT(trace_row, 8 * h + 4, it);
+      FA2_TRACE_AT(trace_row, 8 * g + 4, it);
       tc_fence_after();
       float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i_first + it) * C::BM) * D;
-      if (C::DQ_T) {
-        // lane r holds dQ^T[d = r][query 64h + q]: each warp instruction adds 32
+      if constexpr (C::DQ_T) {
+        // lane r holds dQ^T[d = r][query CW g + q]: each warp instruction adds 32
         // consecutive d values of one query row (128 contiguous bytes)
-        float v[64];
-        tmem_ld64(lane_base + C::COL_DQ + 64 * h, v);
+        float v[CW];
+        tmem_ld32(lane_base + C::COL_DQ + CW * g, v);
         tc_fence_before();
         mbar_arrive(bar_dq_empty);
-        float* col = acc + static_cast<size_t>(64 * h) * D + r;
+        float* col = acc + static_cast<size_t>(CW * g) * D + r;
 #pragma unroll
-        for (int q = 0; q < 64; ++q) red_add(col + static_cast<size_t>(q) * D, v[q]);
+        for (int q = 0; q < CW; ++q) red_add(col + static_cast<size_t>(q) * D, v[q]);
       } else {
-        // lane r holds dQ[query r][d]; this half adds d columns [h D/2, (h+1) D/2)
-        float v[D / 2];
-        if constexpr (D == 128)
-          tmem_ld64(lane_base + C::COL_DQ + (D / 2) * h, v);
+        // lane r holds dQ[query r][d]; this group adds d columns [g D/4, (g+1) D/4)
+        constexpr int DW = D / C::NWG;
+        float v[DW];
+        if constexpr (DW == 32)
+          tmem_ld32(lane_base + C::COL_DQ + DW * g, v);
         else
-          tmem_ld32(lane_base + C::COL_DQ + (D / 2) * h, v);
+          tmem_ld16(lane_base + C::COL_DQ + DW * g, v);
         tc_fence_before();
         mbar_arrive(bar_dq_empty);
-        float* row = acc + static_cast<size_t>(r) * D + (D / 2) * h;
+        float* row = acc + static_cast<size_t>(r) * D + DW * g;
 #pragma unroll
-        for (int e = 0; e < D / 2; e += 4) red_add_v4(row + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
+        for (int e = 0; e < DW; e += 4) red_add_v4(row + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
       }
-      FA2_TRACE_AT(trace_row, 8 * h + 5, it);
+      FA2_TRACE_AT(trace_row, 8 * g + 5, it);
       return true;
     };
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int i = i_first + it;
       const int s = it % C::STAGES;
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 2 * C::VEC_BYTES) + 64 * h;
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 2 * C::VEC_BYTES) + CW * g;
       const float* dlt = lse2 + 128;
-      FA2_TRACE_AT(trace_row, 8 * h + 0, it);
+      FA2_TRACE_AT(trace_row, 8 * g + 0, it);
       // LSE2 and D of this query block were written by the TMA (async proxy)
       ok = mbar_wait(bar_st_full(s), (it / C::STAGES) & 1, abort_flag, 0x1300);
       if (!ok) break;
       ok = mbar_wait(bar_s_full, it & 1, abort_flag, 0x1301);
       if (!ok) break;
-      FA2_TRACE_AT(trace_row, 8 * h + 1, it);
+      FA2_TRACE_AT(trace_row, 8 * g + 1, it);
       tc_fence_after();
-      // P^T for query columns [64h, 64h + 64)
-      uint32_t pk[32];
+      // P^T for query columns [CW g, CW g + CW)
+      uint32_t pk[CW / 2];
       {
-        float sv[64];
-        tmem_ld64(lane_base + C::COL_S + 64 * h, sv);
+        float sv[CW];
+        tmem_ld32(lane_base + C::COL_S + CW * g, sv);
         const unsigned long long c2 = f2(c, c);
         const bool diag = p.causal && (i == ktile);
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) {
+        for (int e = 0; e < CW; e += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2 + e);
           float x0, x1, x2, x3;
           f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
           f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
           float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
           if (diag) {  // query i*128 + q sees key k0 + r only if q >= r
-            const int q = 64 * h + e;
+            const int q = CW * g + e;
             if (q < r) p0 = 0.f;
             if (q + 1 < r) p1 = 0.f;
             if (q + 2 < r) p2 = 0.f;
@@ -491,12 +499,12 @@ __global__ void __launch_bounds__(320, 1)
           pk[e / 2 + 1] = pack_bf16(p2, p3);
         }
       }
-      // P^T over this half's own first 32 S^T columns (already read above)
-      tmem_st32(lane_base + C::COL_S + 64 * h, pk);
+      // P^T over the group's own first CW/2 S^T columns (already read above)
+      tmem_st16(lane_base + C::COL_S + CW * g, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_ready);
-      FA2_TRACE_AT(trace_row, 8 * h + 2, it);
+      FA2_TRACE_AT(trace_row, 8 * g + 2, it);
       // the previous step's dQ is ready by now (its MMAs ran while P^T was formed)
       if (it > 0) {
         ok = drain(it - 1);
@@ -506,17 +514,22 @@ __global__ void __launch_bounds__(320, 1)
       ok = mbar_wait(bar_dp_full, it & 1, abort_flag, 0x1302);
       if (!ok) break;
       tc_fence_after();
-      uint32_t dk[32];
+      uint32_t dk[CW / 2];
       {
-        float dp[64];
-        tmem_ld64(lane_base + C::COL_DP + 64 * h, dp);
+        float dp[CW];
+        tmem_ld32(lane_base + C::COL_DP + CW * g, dp);
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) {
+        for (int e = 0; e < CW; e += 4) {
           const float4 d4 = *reinterpret_cast<const float4*>(dlt + e);
-          const float p0 = __uint_as_float(pk[e / 2] << 16), p1 = __uint_as_float(pk[e / 2] & 0xFFFF0000u);
-          const float p2 = __uint_as_float(pk[e / 2 + 1] << 16), p3 = __uint_as_float(pk[e / 2 + 1] & 0xFFFF0000u);
-          dk[e / 2] = pack_bf16(p0 * (dp[e] - d4.x), p1 * (dp[e + 1] - d4.y));
-          dk[e / 2 + 1] = pack_bf16(p2 * (dp[e + 2] - d4.z), p3 * (dp[e + 3] - d4.w));
+          const unsigned long long pa = f2(__uint_as_float(pk[e / 2] << 16), __uint_as_float(pk[e / 2] & 0xFFFF0000u));
+          const unsigned long long pb = f2(__uint_as_float(pk[e / 2 + 1] << 16), __uint_as_float(pk[e / 2 + 1] & 0xFFFF0000u));
+          const unsigned long long da = f2_add(f2(dp[e], dp[e + 1]), f2(-d4.x, -d4.y));
+          const unsigned long long db = f2_add(f2(dp[e + 2], dp[e + 3]), f2(-d4.z, -d4.w));
+          float s0, s1, s2, s3;
+          f2_split(f2_mul(pa, da), s0, s1);
+          f2_split(f2_mul(pb, db), s2, s3);
+          dk[e / 2] = pack_bf16(s0, s1);
+          dk[e / 2 + 1] = pack_bf16(s2, s3);
         }
       }
       if (it > 0) {  // dK_{i-1} and dQ_{i-1} have finished reading the dS^T tile
@@ -524,44 +537,47 @@ __global__ void __launch_bounds__(320, 1)
         if (!ok) break;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t off = sw128_offset(r, 8 * h + u);
+      for (int u = 0; u < CW / 8; ++u) {
+        const uint32_t off = sw128_offset(r, (CW / 8) * g + u);
         *reinterpret_cast<uint4*>(ds_base + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
       }
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(bar_ds_ready);
-      FA2_TRACE_AT(trace_row, 8 * h + 3, it);
+      FA2_TRACE_AT(trace_row, 8 * g + 3, it);
     }
     if (ok && n_iter > 0) ok = drain(n_iter - 1);
     if (ok) ok = mbar_wait(bar_dkv_done, 0, abort_flag, 0x1305);
     if (ok) {
-      // epilogue: this half stores d columns [h D/2, (h+1) D/2) of dV and scale * dK
+      // epilogue: group g stores d columns [g D/4, (g+1) D/4) of dV and scale * dK
+      constexpr int DW = D / C::NWG;
       tc_fence_after();
       const bool store = key < p.N;
-      const size_t off = (static_cast<size_t>(bh) * p.N + key) * D;
-#pragma unroll 1
-      for (int q = 0; q < D / 64; ++q) {
-        const int c0 = h * (D / 2) + 32 * q;
-        float v[32];
-        uint4 w[4];
-        uint32_t* wu = reinterpret_cast<uint32_t*>(w);
-        tmem_ld32(lane_base + C::COL_DV + c0, v);
+      const size_t off = (static_cast<size_t>(bh) * p.N + key) * D + DW * g;
+      float v[DW];
+      uint4 w[DW / 8];
+      uint32_t* wu = reinterpret_cast<uint32_t*>(w);
+      if constexpr (DW == 32)
+        tmem_ld32(lane_base + C::COL_DV + DW * g, v);
+      else
+        tmem_ld16(lane_base + C::COL_DV + DW * g, v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) wu[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dv + off + c0);
+      for (int e = 0; e < DW / 2; ++e) wu[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+      if (store) {
+        uint4* dst = reinterpret_cast<uint4*>(p.dv + off);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = w[e];
-        }
-        tmem_ld32(lane_base + C::COL_DK + c0, v);
+        for (int e = 0; e < DW / 8; ++e) dst[e] = w[e];
+      }
+      if constexpr (DW == 32)
+        tmem_ld32(lane_base + C::COL_DK + DW * g, v);
+      else
+        tmem_ld16(lane_base + C::COL_DK + DW * g, v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) wu[e] = pack_bf16(v[2 * e] * p.scale, v[2 * e + 1] * p.scale);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dk + off + c0);
+      for (int e = 0; e < DW / 2; ++e) wu[e] = pack_bf16(v[2 * e] * p.scale, v[2 * e + 1] * p.scale);
+      if (store) {
+        uint4* dst = reinterpret_cast<uint4*>(p.dk + off);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = w[e];
-        }
+        for (int e = 0; e < DW / 8; ++e) dst[e] = w[e];
       }
     }
   }
@@ -569,7 +585,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == C::WARP_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fa2
