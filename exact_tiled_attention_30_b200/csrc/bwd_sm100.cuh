@@ -322,14 +322,24 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);      // dV, dK
       constexpr uint32_t IDESC_QT = idesc_bf16(128, 128, true, true);     // dQ^T (d = 128)
       constexpr uint32_t IDESC_Q = idesc_bf16(128, D, true, true);        // dQ (d = 64)
+      // descriptor halves of every operand buffer, built once
+      const SDesc dK = sdesc_make(sbase + C::OFF_K, 16, 1024);                // K-major
+      const SDesc dV = sdesc_make(sbase + C::OFF_V, 16, 1024);
+      const SDesc dQk = sdesc_make(sbase + C::OFF_Q, 16, 1024);
+      const SDesc dOk = sdesc_make(sbase + C::OFF_DO, 16, 1024);
+      const SDesc dQm = sdesc_make(sbase + C::OFF_Q, C::CHUNK_BYTES, 1024);   // MN-major
+      const SDesc dOm = sdesc_make(sbase + C::OFF_DO, C::CHUNK_BYTES, 1024);
+      const SDesc dKm = sdesc_make(sbase + C::OFF_K, C::CHUNK_BYTES, 1024);
+      const SDesc dSk = sdesc_make(sbase + C::OFF_DS, 16, 1024);
+      const SDesc dSm = sdesc_make(sbase + C::OFF_DS, C::CHUNK_BYTES, 1024);
+      constexpr uint32_t TILE16 = C::TILE_BYTES / 16;  // stage stride in descriptor units
+      auto kmaj = [](int k) -> uint32_t { return ((k >> 2) * C::CHUNK_BYTES + (k & 3) * 32) >> 4; };
       auto issue_s = [&](int it) {  // S^T = K Q_i^T
-        const uint32_t q_s = sbase + C::OFF_Q + (it % C::STAGES) * C::TILE_BYTES;
+        const uint32_t qlo = dQk.lo + (it % C::STAGES) * TILE16;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
-          umma_ss(tmem + C::COL_S, sdesc_sw128(sbase + C::OFF_K + off, 16, 1024),
-                  sdesc_sw128(q_s + off, 16, 1024), IDESC_SS, k > 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < D / 16; ++k)
+          umma_ss2(tmem + C::COL_S, dK.lo + kmaj(k), dK.hi, qlo + kmaj(k), dQk.hi, IDESC_SS,
+                   k > 0 ? 1u : 0u);
         umma_commit(bar_s_full);
       };
       bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x1201) &&
@@ -343,8 +353,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // core runs dK_i and dQ_i; it overwrites P^T_i only after dV_i in issue order.
       for (int it = 0; it < n_iter && ok; ++it) {
         const int s = it % C::STAGES;
-        const uint32_t q_s = sbase + C::OFF_Q + s * C::TILE_BYTES;
-        const uint32_t do_s = sbase + C::OFF_DO + s * C::TILE_BYTES;
+        const uint32_t acc0 = it > 0 ? 1u : 0u;
         FA2_TRACE_AT(trace_cta, 16, it);
         if (C::DQ_IN_DP && it > 0) {  // the dP^T columns hold dQ_{i-1} until it is read out
           ok = mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x1203);
@@ -352,25 +361,24 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           tc_fence_after();
         }
         FA2_TRACE_AT(trace_cta, 17, it);
+        const uint32_t dolo = dOk.lo + s * TILE16;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {  // dP^T = V dO_i^T
-          const uint32_t off = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
-          umma_ss(tmem + C::COL_DP, sdesc_sw128(sbase + C::OFF_V + off, 16, 1024),
-                  sdesc_sw128(do_s + off, 16, 1024), IDESC_SS, k > 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < D / 16; ++k)  // dP^T = V dO_i^T
+          umma_ss2(tmem + C::COL_DP, dV.lo + kmaj(k), dV.hi, dolo + kmaj(k), dOk.hi, IDESC_SS,
+                   k > 0 ? 1u : 0u);
         umma_commit(bar_dp_full);
-        // dV += P^T dO_i once both halves have written P^T
+        // dV += P^T dO_i once every group has written P^T
         ok = mbar_wait(bar_p_ready, it & 1, abort_flag, 0x1204);
         if (!ok) break;
         FA2_TRACE_AT(trace_cta, 18, it);
         tc_fence_after();
+        const uint32_t domlo = dOm.lo + s * TILE16;
 #pragma unroll
         for (int k = 0; k < C::BM / 16; ++k) {
           // queries 16k..16k+15 sit in group g = 16k / CW at column CW g + (16k mod CW) / 2
           const uint32_t pcol = C::COL_S + C::CW * ((16 * k) / C::CW) + ((16 * k) % C::CW) / 2;
-          umma_ts(tmem + C::COL_DV, tmem + pcol,
-                  sdesc_sw128(do_s + k * 2048, C::CHUNK_BYTES, 1024), IDESC_KV,
-                  (it > 0 || k > 0) ? 1u : 0u);
+          umma_ts2(tmem + C::COL_DV, tmem + pcol, domlo + k * (2048 >> 4), dOm.hi, IDESC_KV,
+                   k > 0 ? 1u : acc0);
         }
         if (it + 1 < n_iter) {
           ok = mbar_wait(bar_st_full((it + 1) % C::STAGES), ((it + 1) / C::STAGES) & 1, abort_flag,
@@ -384,14 +392,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (!ok) break;
         FA2_TRACE_AT(trace_cta, 19, it);
         tc_fence_after();
-        const uint32_t ds = sbase + C::OFF_DS;
+        const uint32_t qmlo = dQm.lo + s * TILE16;
 #pragma unroll
-        for (int k = 0; k < C::BM / 16; ++k) {
-          const uint32_t aoff = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
-          umma_ss(tmem + C::COL_DK, sdesc_sw128(ds + aoff, 16, 1024),
-                  sdesc_sw128(q_s + k * 2048, C::CHUNK_BYTES, 1024), IDESC_KV,
-                  (it > 0 || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < C::BM / 16; ++k)
+          umma_ss2(tmem + C::COL_DK, dSk.lo + kmaj(k), dSk.hi, qmlo + k * (2048 >> 4), dQm.hi,
+                   IDESC_KV, k > 0 ? 1u : acc0);
         if (!C::DQ_IN_DP && it > 0) {  // dQ_{i-1} must be read out before it is overwritten
           ok = mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x1206);
           if (!ok) break;
@@ -399,12 +404,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k) {  // reduction over the 128 keys
-          const uint64_t kdesc = sdesc_sw128(sbase + C::OFF_K + k * 2048, C::CHUNK_BYTES, 1024);
-          const uint64_t sdesc = sdesc_sw128(ds + k * 2048, C::CHUNK_BYTES, 1024);
-          if (C::DQ_T)
-            umma_ss(tmem + C::COL_DQ, kdesc, sdesc, IDESC_QT, k > 0 ? 1u : 0u);  // K^T dS^T
-          else
-            umma_ss(tmem + C::COL_DQ, sdesc, kdesc, IDESC_Q, k > 0 ? 1u : 0u);   // dS K
+          if (C::DQ_T)  // dQ^T = K^T dS^T
+            umma_ss2(tmem + C::COL_DQ, dKm.lo + k * (2048 >> 4), dKm.hi, dSm.lo + k * (2048 >> 4),
+                     dSm.hi, IDESC_QT, k > 0 ? 1u : 0u);
+          else  // dQ = dS K
+            umma_ss2(tmem + C::COL_DQ, dSm.lo + k * (2048 >> 4), dSm.hi, dKm.lo + k * (2048 >> 4),
+                     dKm.hi, IDESC_Q, k > 0 ? 1u : 0u);
         }
         umma_commit(bar_dq_full);
         umma_commit(bar_dsm_free);

@@ -179,26 +179,32 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(128, C::BN, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
+      // descriptor halves of every operand buffer, built once
+      const SDesc dq0 = sdesc_make(sbase + C::OFF_Q, 16, 1024);
+      const SDesc dq1 = sdesc_make(sbase + C::OFF_Q + C::TILE_BYTES, 16, 1024);
+      const SDesc dk0 = sdesc_make(sbase + C::OFF_K, 16, 1024);
+      const SDesc dv0 = sdesc_make(sbase + C::OFF_V, C::CHUNK_BYTES, 1024);
+      constexpr uint32_t STAGE16 = 2 * C::TILE_BYTES / 16;  // stage stride in descriptor units
       auto issue_s = [&](int t, int j) {
-        const uint32_t kbase = sbase + C::OFF_K + (j % C::STAGES) * 2 * C::TILE_BYTES;
-        const uint32_t qbase = sbase + C::OFF_Q + t * C::TILE_BYTES;
+        const uint32_t klo = dk0.lo + (j % C::STAGES) * STAGE16;
+        const uint32_t qlo = t ? dq1.lo : dq0.lo;
+        const uint32_t dcol = tmem + (t ? C::COL_S1 : C::COL_S0);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
-          umma_ss(tmem + (t ? C::COL_S1 : C::COL_S0), sdesc_sw128(qbase + off, 16, 1024),
-                  sdesc_sw128(kbase + off, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
+          const uint32_t off = ((k >> 2) * C::CHUNK_BYTES + (k & 3) * 32) >> 4;
+          umma_ss2(dcol, qlo + off, dq0.hi, klo + off, dk0.hi, IDESC_S, k > 0 ? 1u : 0u);
         }
         umma_commit(bar_s_full(t));
       };
       auto issue_pv = [&](int t, int j) {
-        const uint32_t vbase = sbase + C::OFF_V + (j % C::STAGES) * 2 * C::TILE_BYTES;
+        const uint32_t vlo = dv0.lo + (j % C::STAGES) * STAGE16;
         const uint32_t pcol = tmem + (t ? C::COL_S1 : C::COL_S0);
         const uint32_t ocol = tmem + (t ? C::COL_O1 : C::COL_O0);
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k) {
           // V: MN-major (d contiguous), 16 keys = 2 swizzle atoms of 8 rows
-          umma_ts(ocol, pcol + k * 8, sdesc_sw128(vbase + k * 16 * 128, C::CHUNK_BYTES, 1024),
-                  IDESC_O, (j > 0 || k > 0) ? 1u : 0u);
+          umma_ts2(ocol, pcol + k * 8, vlo + k * (2048 >> 4), dv0.hi, IDESC_O, k > 0 ? 1u : acc0);
         }
       };
       bool ok = mbar_wait(bar_q, 0, abort_flag, 0x201) &&
