@@ -247,6 +247,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
+  FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 30, 0);
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
     for (int s = 0; s < C::STAGES; ++s) {
@@ -279,6 +280,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 31, 0);
 
   if (warp == C::WARP_TMA) {
     // ------------------------------------------------------------ TMA producer
@@ -553,6 +555,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     if (ok && n_iter > 0) ok = drain(n_iter - 1);
     if (ok) ok = mbar_wait(bar_dkv_done, 0, abort_flag, 0x1305);
+    FA2_TRACE_AT(trace_row, 32, 0);
     if (ok) {
       // epilogue: group g stores d columns [g D/4, (g+1) D/4) of dV and scale * dK
       constexpr int DW = D / C::NWG;
@@ -590,6 +593,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 33, 0);
   if (warp == C::WARP_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
