@@ -13,7 +13,7 @@
 // Kernels, all on the caller's stream:
 //   1. fa2_bwd_pre: D and LSE * log2(e) into the workspace (rows padded to a
 //      multiple of 128: D = 0, LSE = +inf there so P vanishes), dQ accumulator
-//      zeroed. HBM-bound.
+//      and the main kernel's work-item counter zeroed. HBM-bound.
 //   2. fa2_bwd_kernel: one CTA per (128-key block, batch*head), parallel over key
 //      blocks; dK and dV accumulate in tensor memory over all query blocks, dQ
 //      is added into an fp32 accumulator with reductions (layout below).
@@ -32,6 +32,7 @@ struct BwdPreParams {
   float* dq_acc;   // [BH][Np][d]
   float* delta;    // [BH][Np]
   float* lse2;     // [BH][Np]
+  unsigned int* counter;  // work-item counter of the main kernel
   int N;
   int Np;
   long long rows;  // BH * Np
@@ -43,6 +44,7 @@ __global__ void __launch_bounds__(256) fa2_bwd_pre_kernel(const BwdPreParams p) 
   constexpr int TPR = D / 8;            // threads per row
   constexpr int RPB = 256 / TPR;        // rows per block per sweep
   const int sub = threadIdx.x % TPR;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.counter = 0u;
   const long long stride = static_cast<long long>(gridDim.x) * RPB;
   for (long long r = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / TPR; r < p.rows;
        r += stride) {
@@ -111,9 +113,13 @@ __global__ void __launch_bounds__(256) fa2_bwd_dq_convert_kernel(const BwdConver
 
 
 // ------------------------------------------------------------ main kernel (B2)
-// One CTA per (128-key block j, batch*head); query blocks i stream through a
-// two-stage TMA ring (causal: only i >= j, the diagonal block first).
-//   warp 16       TMA producer: K_j, V_j once; Q_i, dO_i, LSE2_i, D_i per step
+// Persistent: one CTA per SM takes work items (128-key block j, batch*head)
+// from a counter in the workspace, longest first within groups of heads
+// (causal: low j sees the most query blocks). Per item, query blocks i stream
+// through a two-stage TMA ring (causal: only i >= j, the diagonal block first).
+//   warp 16       TMA producer and scheduler: fetches the next item, hands it to
+//                 the other warps through a two-slot ring, loads K_j, V_j once the
+//                 previous item's MMAs are done, then Q_i, dO_i, LSE2_i, D_i
 //   warp 17       MMA issuer + TMEM owner, per step:
 //                   S^T = K Q_i^T,  dP^T = V dO_i^T          (keys on TMEM lanes)
 //                   dV += P^T dO_i    (P^T from TMEM)
@@ -121,20 +127,24 @@ __global__ void __launch_bounds__(256) fa2_bwd_dq_convert_kernel(const BwdConver
 //                   d = 128: dQ^T = K^T dS^T (d on lanes; dS^T read MN-major)
 //                   d =  64: dQ   = dS K     (queries on lanes)
 //   warps 0-15    four elementwise warpgroups; warpgroup g owns query columns
-//                 [32g, 32g + 32) of the step and thread r key row r. P^T =
+//                 [32g, 32g + 32) of a step and thread r key row r. P^T =
 //                 exp2(c S^T - LSE2) goes back into TMEM over the group's own
 //                 S^T columns; dS^T = P^T (dP^T - D) goes to swizzled smem; then
 //                 the group adds its share of dQ into the fp32 accumulator with
 //                 reductions. No row statistics are needed (P comes from the
-//                 saved LSE), so the groups never exchange data.
+//                 saved LSE), so the groups never exchange data. After an item's
+//                 last step they store dK, dV, while the MMA warp already starts
+//                 the next item.
 // Tensor memory: S^T [0,128) (P^T of group g in [32g, 32g+16)), dP^T [128,256),
 // dV [256,256+D), dK [256+D,256+2D); dQ^T (d = 128) reuses the dP^T columns once
 // dS is in smem, dQ (d = 64) has [384,448).
+// Every barrier phase is counted over the whole sequence of items: `gs` counts
+// steps, `n` counts items.
 template <int D>
 struct BwdCfg {
   static_assert(D == 64 || D == 128, "head dim");
   static constexpr int BM = 128;                      // query rows per step
-  static constexpr int BN = 128;                      // keys per CTA
+  static constexpr int BN = 128;                      // keys per item
   static constexpr int STAGES = 2;
   static constexpr int CHUNKS = D / 64;
   static constexpr int TILE_BYTES = 128 * D * 2;
@@ -147,10 +157,11 @@ struct BwdCfg {
   static constexpr int OFF_DS = OFF_DO + STAGES * TILE_BYTES;     // 128 x 128 bf16
   static constexpr int OFF_VEC = OFF_DS + 32768;                  // [s][LSE2 | D]
   static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
-  // kv_full, st_full[S], st_empty[S], s_full, dp_full, p_ready, ds_ready,
-  // dsm_free, dq_full, dq_empty, dkv_done, drain
-  static constexpr int NUM_BARS = 1 + 2 * STAGES + 9;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
+  // kv_full, kv_empty, st_full[S], st_empty[S], s_full, dp_full, p_ready,
+  // ds_ready, dsm_free, dq_full, dq_empty, dkv_done, dkv_free, drain,
+  // item_full[2], item_empty[2]
+  static constexpr int NUM_BARS = 2 + 2 * STAGES + 10 + 4;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;         // tmem slot, abort, items[2]
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   // d = 128 uses 231,6xx bytes: there is no room for alignment slack, so the
   // kernel checks that the dynamic shared memory base is 1024-byte aligned
@@ -171,16 +182,19 @@ struct BwdCfg {
   // d = 128 has no free columns left: dQ reuses the dP^T columns once dS is in smem
   static constexpr bool DQ_IN_DP = (D == 128);
   static constexpr uint32_t COL_DQ = DQ_IN_DP ? COL_DP : 256 + 2 * D;
+  static constexpr int HEAD_GROUP = 16;               // heads per scheduling group
 };
 
 struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  float* dq_acc;       // [BH][Np][d]
-  const float* lse2;   // [BH][Np]
-  const float* delta;  // [BH][Np]
+  float* dq_acc;          // [BH][Np][d]
+  const float* lse2;      // [BH][Np]
+  const float* delta;     // [BH][Np]
+  unsigned int* counter;  // next work item (zeroed by the preprocess kernel)
   int N;
   int Np;
+  int BH;
   int n_ktiles;
   int causal;
   float scale;
@@ -203,6 +217,26 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int u) {
   return static_cast<uint32_t>((u >> 3) * 16384 + r * 128 + (((u & 7) ^ (r & 7)) << 4));
 }
 
+// Work item -> (key tile, batch*head). Non-causal items all cost the same: the
+// key tiles of one head are consecutive, so they run together and share the
+// head's Q/dO in L2. Causal items come in groups of HEAD_GROUP heads (their Q/dO
+// stay in L2 while the group runs); inside a group the key tile is the slow
+// index, so the items with the most query blocks come first.
+__device__ __forceinline__ void decode_item(int item, int n_ktiles, int BH, int head_group,
+                                            bool causal, int& ktile, int& bh) {
+  if (!causal) {
+    bh = item / n_ktiles;
+    ktile = item - bh * n_ktiles;
+    return;
+  }
+  const int group_items = head_group * n_ktiles;
+  const int grp = item / group_items;
+  const int r = item - grp * group_items;
+  const int heads = min(head_group, BH - grp * head_group);
+  ktile = r / heads;
+  bh = grp * head_group + (r - ktile * heads);
+}
+
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -219,23 +253,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // grid (key tile, batch*head): the key blocks of one head run together and
-  // share its Q/dO tiles in L2 (measured faster than a longest-first order
-  // across heads, even for causal masks)
-  const int ktile = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int k0 = ktile * C::BN;
-  const int n_qtiles = p.n_ktiles;  // self-attention: same N
-  const int i_first = p.causal ? ktile : 0;
-  const int n_iter = n_qtiles - i_first;
+  const int n_items = p.n_ktiles * p.BH;
 #ifdef FA2_TRACE
-  const bool trace_cta = blockIdx.x == 0 && blockIdx.y == 7;
+  const bool trace_cta = blockIdx.x == 7;
 #endif
 
-  const uint32_t bar_kv = sbase + C::OFF_BAR;
-  auto bar_st_full = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + s); };
-  auto bar_st_empty = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + C::STAGES + s); };
-  const uint32_t bar_s_full = sbase + C::OFF_BAR + 8 * (1 + 2 * C::STAGES);
+  const uint32_t bar_kv_full = sbase + C::OFF_BAR;
+  const uint32_t bar_kv_empty = bar_kv_full + 8;
+  auto bar_st_full = [&](int s) { return sbase + C::OFF_BAR + 8 * (2 + s); };
+  auto bar_st_empty = [&](int s) { return sbase + C::OFF_BAR + 8 * (2 + C::STAGES + s); };
+  const uint32_t bar_s_full = sbase + C::OFF_BAR + 8 * (2 + 2 * C::STAGES);
   const uint32_t bar_dp_full = bar_s_full + 8;
   const uint32_t bar_p_ready = bar_s_full + 16;
   const uint32_t bar_ds_ready = bar_s_full + 24;
@@ -243,13 +270,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const uint32_t bar_dq_full = bar_s_full + 40;
   const uint32_t bar_dq_empty = bar_s_full + 48;
   const uint32_t bar_dkv_done = bar_s_full + 56;
-  const uint32_t bar_drain = bar_s_full + 64;
+  const uint32_t bar_dkv_free = bar_s_full + 64;
+  const uint32_t bar_drain = bar_s_full + 72;
+  auto bar_item_full = [&](int q) { return bar_s_full + 80 + 8 * q; };
+  auto bar_item_empty = [&](int q) { return bar_s_full + 96 + 8 * q; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
 
   FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 30, 0);
   if (threadIdx.x == 0) {
-    mbar_init(bar_kv, 1);
+    mbar_init(bar_kv_full, 1);
+    mbar_init(bar_kv_empty, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(bar_st_full(s), 1);
       mbar_init(bar_st_empty(s), 1);
@@ -262,7 +294,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_init(bar_dq_full, 1);
     mbar_init(bar_dq_empty, C::ELEM_THREADS);
     mbar_init(bar_dkv_done, 1);
+    mbar_init(bar_dkv_free, C::ELEM_THREADS);
     mbar_init(bar_drain, 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(bar_item_full(q), 1);
+      mbar_init(bar_item_empty(q), 1 + C::ELEM_THREADS);  // MMA thread + elementwise threads
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -282,40 +319,71 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 31, 0);
 
+  // Consumers read item n from the two-slot ring (-1 ends the sequence).
+  auto take_item = [&](int n, int site) -> int {
+    if (!mbar_wait(bar_item_full(n & 1), (n >> 1) & 1, abort_flag, site)) return -1;
+    const int item = item_slot[n & 1];
+    mbar_arrive(bar_item_empty(n & 1));
+    return item;
+  };
+  auto steps_of = [&](int ktile) { return p.causal ? p.n_ktiles - ktile : p.n_ktiles; };
+
   if (warp == C::WARP_TMA) {
-    // ------------------------------------------------------------ TMA producer
+    // --------------------------------------------------- scheduler + TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
-      for (int c = 0; c < C::CHUNKS; ++c) {
-        tma_load_3d(sbase + C::OFF_K + c * C::CHUNK_BYTES, &tm_k, bar_kv, c * 64, k0, bh);
-        tma_load_3d(sbase + C::OFF_V + c * C::CHUNK_BYTES, &tm_v, bar_kv, c * 64, k0, bh);
-      }
-      int last_parity[C::STAGES];
-      for (int s = 0; s < C::STAGES; ++s) last_parity[s] = -1;
+      int last_st_parity[C::STAGES];
+      for (int s = 0; s < C::STAGES; ++s) last_st_parity[s] = -1;
+      int last_kv_parity = -1;
       bool ok = true;
-      for (int it = 0; it < n_iter && ok; ++it) {
-        const int i = i_first + it;
-        const int s = it % C::STAGES;
-        const int n = it / C::STAGES;
-        if (n > 0) ok = mbar_wait(bar_st_empty(s), (n - 1) & 1, abort_flag, 0x1101);
+      int gs = 0;
+      for (int n = 0; ok; ++n) {
+        int item = static_cast<int>(atomicAdd(p.counter, 1u));
+        if (item >= n_items) item = -1;
+        if (n >= 2) ok = mbar_wait(bar_item_empty(n & 1), ((n >> 1) - 1) & 1, abort_flag, 0x1100);
         if (!ok) break;
-        const uint32_t bar = bar_st_full(s);
-        mbar_arrive_expect_tx(bar, 2 * C::TILE_BYTES + 2 * C::VEC_BYTES);
-        for (int c = 0; c < C::CHUNKS; ++c) {
-          tma_load_3d(sbase + C::OFF_Q + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar, c * 64,
-                      i * C::BM, bh);
-          tma_load_3d(sbase + C::OFF_DO + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do, bar,
-                      c * 64, i * C::BM, bh);
+        item_slot[n & 1] = item;
+        mbar_arrive(bar_item_full(n & 1));
+        if (item < 0) break;
+        int ktile, bh;
+        decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
+        const int i_first = p.causal ? ktile : 0;
+        const int n_iter = steps_of(ktile);
+        for (int it = 0; it < n_iter && ok; ++it, ++gs) {
+          const int i = i_first + it;
+          const int s = gs % C::STAGES;
+          if (gs >= C::STAGES) ok = mbar_wait(bar_st_empty(s), ((gs / C::STAGES) - 1) & 1, abort_flag, 0x1101);
+          if (!ok) break;
+          if (it == 1 || n_iter == 1) {
+            // K_j, V_j (after the first step's Q/dO is on its way) once the
+            // previous item's MMAs are done with the buffers
+            if (n >= 1) ok = mbar_wait(bar_kv_empty, (n - 1) & 1, abort_flag, 0x1104);
+            if (!ok) break;
+            mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE_BYTES);
+            for (int c = 0; c < C::CHUNKS; ++c) {
+              tma_load_3d(sbase + C::OFF_K + c * C::CHUNK_BYTES, &tm_k, bar_kv_full, c * 64, ktile * C::BN, bh);
+              tma_load_3d(sbase + C::OFF_V + c * C::CHUNK_BYTES, &tm_v, bar_kv_full, c * 64, ktile * C::BN, bh);
+            }
+            last_kv_parity = n & 1;
+          }
+          const uint32_t bar = bar_st_full(s);
+          mbar_arrive_expect_tx(bar, 2 * C::TILE_BYTES + 2 * C::VEC_BYTES);
+          for (int c = 0; c < C::CHUNKS; ++c) {
+            tma_load_3d(sbase + C::OFF_Q + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar,
+                        c * 64, i * C::BM, bh);
+            tma_load_3d(sbase + C::OFF_DO + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do, bar,
+                        c * 64, i * C::BM, bh);
+          }
+          const size_t voff = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * C::BM;
+          const uint32_t vec = sbase + C::OFF_VEC + s * 2 * C::VEC_BYTES;
+          bulk_load(vec, p.lse2 + voff, C::VEC_BYTES, bar);
+          bulk_load(vec + C::VEC_BYTES, p.delta + voff, C::VEC_BYTES, bar);
+          last_st_parity[s] = (gs / C::STAGES) & 1;
         }
-        const size_t voff = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * C::BM;
-        const uint32_t vec = sbase + C::OFF_VEC + s * 2 * C::VEC_BYTES;
-        bulk_load(vec, p.lse2 + voff, C::VEC_BYTES, bar);
-        bulk_load(vec + C::VEC_BYTES, p.delta + voff, C::VEC_BYTES, bar);
-        last_parity[s] = n & 1;
       }
-      mbar_wait(bar_kv, 0, abort_flag, 0x1102);
+      // never leave the CTA with copies still landing in its shared memory
+      if (last_kv_parity >= 0) mbar_wait(bar_kv_full, last_kv_parity, abort_flag, 0x1102);
       for (int s = 0; s < C::STAGES; ++s)
-        if (last_parity[s] >= 0) mbar_wait(bar_st_full(s), last_parity[s], abort_flag, 0x1103);
+        if (last_st_parity[s] >= 0) mbar_wait(bar_st_full(s), last_st_parity[s], abort_flag, 0x1103);
     }
   } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
@@ -336,88 +404,103 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const SDesc dSm = sdesc_make(sbase + C::OFF_DS, C::CHUNK_BYTES, 1024);
       constexpr uint32_t TILE16 = C::TILE_BYTES / 16;  // stage stride in descriptor units
       auto kmaj = [](int k) -> uint32_t { return ((k >> 2) * C::CHUNK_BYTES + (k & 3) * 32) >> 4; };
-      auto issue_s = [&](int it) {  // S^T = K Q_i^T
-        const uint32_t qlo = dQk.lo + (it % C::STAGES) * TILE16;
+      auto issue_s = [&](int g) {  // S^T = K Q_i^T for global step g
+        const uint32_t qlo = dQk.lo + (g % C::STAGES) * TILE16;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           umma_ss2(tmem + C::COL_S, dK.lo + kmaj(k), dK.hi, qlo + kmaj(k), dQk.hi, IDESC_SS,
                    k > 0 ? 1u : 0u);
         umma_commit(bar_s_full);
       };
-      bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x1201) &&
-                mbar_wait(bar_st_full(0), 0, abort_flag, 0x1202);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-      }
-      // Per step i: dP^T_i, dV_i, S^T_{i+1}, dK_i, dQ_i. S^T_{i+1} goes right after
-      // dV_i so that the elementwise warps can form P^T_{i+1} while the tensor
-      // core runs dK_i and dQ_i; it overwrites P^T_i only after dV_i in issue order.
-      for (int it = 0; it < n_iter && ok; ++it) {
-        const int s = it % C::STAGES;
-        const uint32_t acc0 = it > 0 ? 1u : 0u;
-        FA2_TRACE_AT(trace_cta, 16, it);
-        if (C::DQ_IN_DP && it > 0) {  // the dP^T columns hold dQ_{i-1} until it is read out
-          ok = mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x1203);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        FA2_TRACE_AT(trace_cta, 17, it);
-        const uint32_t dolo = dOk.lo + s * TILE16;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)  // dP^T = V dO_i^T
-          umma_ss2(tmem + C::COL_DP, dV.lo + kmaj(k), dV.hi, dolo + kmaj(k), dOk.hi, IDESC_SS,
-                   k > 0 ? 1u : 0u);
-        umma_commit(bar_dp_full);
-        // dV += P^T dO_i once every group has written P^T
-        ok = mbar_wait(bar_p_ready, it & 1, abort_flag, 0x1204);
+      bool ok = true;
+      int gs = 0;
+      for (int n = 0; ok; ++n) {
+        const int item = take_item(n, 0x1209);
+        if (item < 0) break;
+        int ktile, bh;
+        decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
+        const int n_iter = steps_of(ktile);
+        ok = mbar_wait(bar_kv_full, n & 1, abort_flag, 0x1201) &&
+             mbar_wait(bar_st_full(gs % C::STAGES), (gs / C::STAGES) & 1, abort_flag, 0x1202);
         if (!ok) break;
-        FA2_TRACE_AT(trace_cta, 18, it);
         tc_fence_after();
-        const uint32_t domlo = dOm.lo + s * TILE16;
+        // S^T of the item's first step: the elementwise warps read the previous
+        // S^T before its p_ready, and its P^T is read by a dV issued earlier
+        issue_s(gs);
+        for (int it = 0; it < n_iter && ok; ++it) {
+          const int g = gs + it;
+          const int s = g % C::STAGES;
+          const uint32_t acc0 = it > 0 ? 1u : 0u;
+          FA2_TRACE_AT(trace_cta && n == 0, 16, it);
+          if (C::DQ_IN_DP && g > 0) {  // the dP^T columns hold dQ of step g-1 until read out
+            ok = mbar_wait(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1203);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          FA2_TRACE_AT(trace_cta && n == 0, 17, it);
+          const uint32_t dolo = dOk.lo + s * TILE16;
 #pragma unroll
-        for (int k = 0; k < C::BM / 16; ++k) {
-          // queries 16k..16k+15 sit in group g = 16k / CW at column CW g + (16k mod CW) / 2
-          const uint32_t pcol = C::COL_S + C::CW * ((16 * k) / C::CW) + ((16 * k) % C::CW) / 2;
-          umma_ts2(tmem + C::COL_DV, tmem + pcol, domlo + k * (2048 >> 4), dOm.hi, IDESC_KV,
-                   k > 0 ? 1u : acc0);
-        }
-        if (it + 1 < n_iter) {
-          ok = mbar_wait(bar_st_full((it + 1) % C::STAGES), ((it + 1) / C::STAGES) & 1, abort_flag,
-                         0x1208);
+          for (int k = 0; k < D / 16; ++k)  // dP^T = V dO_i^T
+            umma_ss2(tmem + C::COL_DP, dV.lo + kmaj(k), dV.hi, dolo + kmaj(k), dOk.hi, IDESC_SS,
+                     k > 0 ? 1u : 0u);
+          umma_commit(bar_dp_full);
+          // dV += P^T dO_i once every group has written P^T
+          ok = mbar_wait(bar_p_ready, g & 1, abort_flag, 0x1204);
           if (!ok) break;
+          if (it == 0 && n > 0) {  // the previous item's dK, dV have been read out
+            ok = mbar_wait(bar_dkv_free, (n - 1) & 1, abort_flag, 0x120A);
+            if (!ok) break;
+          }
+          FA2_TRACE_AT(trace_cta && n == 0, 18, it);
           tc_fence_after();
-          issue_s(it + 1);
+          const uint32_t domlo = dOm.lo + s * TILE16;
+#pragma unroll
+          for (int k = 0; k < C::BM / 16; ++k) {
+            // queries 16k..16k+15 sit in group g = 16k / CW at column CW g + (16k mod CW) / 2
+            const uint32_t pcol = C::COL_S + C::CW * ((16 * k) / C::CW) + ((16 * k) % C::CW) / 2;
+            umma_ts2(tmem + C::COL_DV, tmem + pcol, domlo + k * (2048 >> 4), dOm.hi, IDESC_KV,
+                     k > 0 ? 1u : acc0);
+          }
+          if (it + 1 < n_iter) {
+            ok = mbar_wait(bar_st_full((g + 1) % C::STAGES), ((g + 1) / C::STAGES) & 1, abort_flag,
+                           0x1208);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(g + 1);
+          }
+          // dK += dS^T Q_i and dQ once dS^T is in smem
+          ok = mbar_wait(bar_ds_ready, g & 1, abort_flag, 0x1205);
+          if (!ok) break;
+          FA2_TRACE_AT(trace_cta && n == 0, 19, it);
+          tc_fence_after();
+          const uint32_t qmlo = dQm.lo + s * TILE16;
+#pragma unroll
+          for (int k = 0; k < C::BM / 16; ++k)
+            umma_ss2(tmem + C::COL_DK, dSk.lo + kmaj(k), dSk.hi, qmlo + k * (2048 >> 4), dQm.hi,
+                     IDESC_KV, k > 0 ? 1u : acc0);
+          if (!C::DQ_IN_DP && g > 0) {  // dQ of step g-1 must be read out before it is overwritten
+            ok = mbar_wait(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1206);
+            if (!ok) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int k = 0; k < C::BN / 16; ++k) {  // reduction over the 128 keys
+            if (C::DQ_T)  // dQ^T = K^T dS^T
+              umma_ss2(tmem + C::COL_DQ, dKm.lo + k * (2048 >> 4), dKm.hi, dSm.lo + k * (2048 >> 4),
+                       dSm.hi, IDESC_QT, k > 0 ? 1u : 0u);
+            else  // dQ = dS K
+              umma_ss2(tmem + C::COL_DQ, dSm.lo + k * (2048 >> 4), dSm.hi, dKm.lo + k * (2048 >> 4),
+                       dKm.hi, IDESC_Q, k > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_dq_full);
+          umma_commit(bar_dsm_free);
+          umma_commit(bar_st_empty(s));
         }
-        // dK += dS^T Q_i and dQ once dS^T is in smem
-        ok = mbar_wait(bar_ds_ready, it & 1, abort_flag, 0x1205);
         if (!ok) break;
-        FA2_TRACE_AT(trace_cta, 19, it);
-        tc_fence_after();
-        const uint32_t qmlo = dQm.lo + s * TILE16;
-#pragma unroll
-        for (int k = 0; k < C::BM / 16; ++k)
-          umma_ss2(tmem + C::COL_DK, dSk.lo + kmaj(k), dSk.hi, qmlo + k * (2048 >> 4), dQm.hi,
-                   IDESC_KV, k > 0 ? 1u : acc0);
-        if (!C::DQ_IN_DP && it > 0) {  // dQ_{i-1} must be read out before it is overwritten
-          ok = mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x1206);
-          if (!ok) break;
-          tc_fence_after();
-        }
-#pragma unroll
-        for (int k = 0; k < C::BN / 16; ++k) {  // reduction over the 128 keys
-          if (C::DQ_T)  // dQ^T = K^T dS^T
-            umma_ss2(tmem + C::COL_DQ, dKm.lo + k * (2048 >> 4), dKm.hi, dSm.lo + k * (2048 >> 4),
-                     dSm.hi, IDESC_QT, k > 0 ? 1u : 0u);
-          else  // dQ = dS K
-            umma_ss2(tmem + C::COL_DQ, dSm.lo + k * (2048 >> 4), dSm.hi, dKm.lo + k * (2048 >> 4),
-                     dKm.hi, IDESC_Q, k > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_dq_full);
-        umma_commit(bar_dsm_free);
-        umma_commit(bar_st_empty(s));
+        umma_commit(bar_dkv_done);  // dK, dV of this item complete
+        umma_commit(bar_kv_empty);  // K_j, V_j no longer read
+        gs += n_iter;
       }
-      umma_commit(bar_dkv_done);
       umma_commit(bar_drain);
       mbar_wait(bar_drain, 0, abort_flag, 0x1207);
     }
@@ -426,167 +509,181 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     constexpr int CW = C::CW;
     const int g = warp >> 2;            // query-column group
     const int r = threadIdx.x & 127;    // TMEM lane: key row (S^T, dP^T, dK, dV)
-    const int key = k0 + r;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float c = p.scale_log2;
     uint8_t* ds_base = smem + C::OFF_DS;
-#ifdef FA2_TRACE
-    const bool trace_row = trace_cta && r == 0 && g < 2;
-#endif
-    // dQ of step it (this group's share) -> fp32 accumulator. The TMEM columns are
-    // released as soon as the values are in registers; the reductions follow.
-    auto drain = [&](int it) -> bool {
-      if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x1304)) return false;
-      FA2_TRACE_AT(trace_row, 8 * g + 4, it);
-      tc_fence_after();
-      float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i_first + it) * C::BM) * D;
-      if constexpr (C::DQ_T) {
-        // lane r holds dQ^T[d = r][query CW g + q]: each warp instruction adds 32
-        // consecutive d values of one query row (128 contiguous bytes)
-        float v[CW];
-        tmem_ld32(lane_base + C::COL_DQ + CW * g, v);
-        tc_fence_before();
-        mbar_arrive(bar_dq_empty);
-        float* col = acc + static_cast<size_t>(CW * g) * D + r;
-#pragma unroll
-        for (int q = 0; q < CW; ++q) red_add(col + static_cast<size_t>(q) * D, v[q]);
-      } else {
-        // lane r holds dQ[query r][d]; this group adds d columns [g D/4, (g+1) D/4)
-        constexpr int DW = D / C::NWG;
-        float v[DW];
-        if constexpr (DW == 32)
-          tmem_ld32(lane_base + C::COL_DQ + DW * g, v);
-        else
-          tmem_ld16(lane_base + C::COL_DQ + DW * g, v);
-        tc_fence_before();
-        mbar_arrive(bar_dq_empty);
-        float* row = acc + static_cast<size_t>(r) * D + DW * g;
-#pragma unroll
-        for (int e = 0; e < DW; e += 4) red_add_v4(row + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
-      }
-      FA2_TRACE_AT(trace_row, 8 * g + 5, it);
-      return true;
-    };
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      const int i = i_first + it;
-      const int s = it % C::STAGES;
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 2 * C::VEC_BYTES) + CW * g;
-      const float* dlt = lse2 + 128;
-      FA2_TRACE_AT(trace_row, 8 * g + 0, it);
-      // LSE2 and D of this query block were written by the TMA (async proxy)
-      ok = mbar_wait(bar_st_full(s), (it / C::STAGES) & 1, abort_flag, 0x1300);
-      if (!ok) break;
-      ok = mbar_wait(bar_s_full, it & 1, abort_flag, 0x1301);
-      if (!ok) break;
-      FA2_TRACE_AT(trace_row, 8 * g + 1, it);
-      tc_fence_after();
-      // P^T for query columns [CW g, CW g + CW)
-      uint32_t pk[CW / 2];
-      {
-        float sv[CW];
-        tmem_ld32(lane_base + C::COL_S + CW * g, sv);
-        const unsigned long long c2 = f2(c, c);
-        const bool diag = p.causal && (i == ktile);
+    int gs = 0;
+    for (int n = 0; ok; ++n) {
+      const int item = take_item(n, 0x1309);
+      if (item < 0) break;
+      int ktile, bh;
+      decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
+      const int i_first = p.causal ? ktile : 0;
+      const int n_iter = steps_of(ktile);
+#ifdef FA2_TRACE
+      const bool trace_row = trace_cta && n == 0 && r == 0 && g < 2;
+#endif
+      // dQ of step it (this group's share) -> fp32 accumulator. The TMEM columns
+      // are released as soon as the values are in registers; the reductions follow.
+      auto drain = [&](int it) -> bool {
+        if (!mbar_wait(bar_dq_full, (gs + it) & 1, abort_flag, 0x1304)) return false;
+        FA2_TRACE_AT(trace_row, 8 * g + 4, it);
+        tc_fence_after();
+        float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i_first + it) * C::BM) * D;
+        if constexpr (C::DQ_T) {
+          // lane r holds dQ^T[d = r][query CW g + q]: each warp instruction adds 32
+          // consecutive d values of one query row (128 contiguous bytes)
+          float v[CW];
+          tmem_ld32(lane_base + C::COL_DQ + CW * g, v);
+          tc_fence_before();
+          mbar_arrive(bar_dq_empty);
+          float* col = acc + static_cast<size_t>(CW * g) * D + r;
 #pragma unroll
-        for (int e = 0; e < CW; e += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + e);
-          float x0, x1, x2, x3;
-          f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
-          f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
-          float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-          if (diag) {  // query i*128 + q sees key k0 + r only if q >= r
-            const int q = CW * g + e;
-            if (q < r) p0 = 0.f;
-            if (q + 1 < r) p1 = 0.f;
-            if (q + 2 < r) p2 = 0.f;
-            if (q + 3 < r) p3 = 0.f;
+          for (int q = 0; q < CW; ++q) red_add(col + static_cast<size_t>(q) * D, v[q]);
+        } else {
+          // lane r holds dQ[query r][d]; this group adds d columns [g D/4, (g+1) D/4)
+          constexpr int DW = D / C::NWG;
+          float v[DW];
+          if constexpr (DW == 32)
+            tmem_ld32(lane_base + C::COL_DQ + DW * g, v);
+          else
+            tmem_ld16(lane_base + C::COL_DQ + DW * g, v);
+          tc_fence_before();
+          mbar_arrive(bar_dq_empty);
+          float* row = acc + static_cast<size_t>(r) * D + DW * g;
+#pragma unroll
+          for (int e = 0; e < DW; e += 4) red_add_v4(row + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+        FA2_TRACE_AT(trace_row, 8 * g + 5, it);
+        return true;
+      };
+      for (int it = 0; it < n_iter; ++it) {
+        const int i = i_first + it;
+        const int gg = gs + it;
+        const int s = gg % C::STAGES;
+        const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 2 * C::VEC_BYTES) + CW * g;
+        const float* dlt = lse2 + 128;
+        FA2_TRACE_AT(trace_row, 8 * g + 0, it);
+        // LSE2 and D of this query block were written by the TMA (async proxy)
+        ok = mbar_wait(bar_st_full(s), (gg / C::STAGES) & 1, abort_flag, 0x1300);
+        if (!ok) break;
+        ok = mbar_wait(bar_s_full, gg & 1, abort_flag, 0x1301);
+        if (!ok) break;
+        FA2_TRACE_AT(trace_row, 8 * g + 1, it);
+        tc_fence_after();
+        // P^T for query columns [CW g, CW g + CW)
+        uint32_t pk[CW / 2];
+        {
+          float sv[CW];
+          tmem_ld32(lane_base + C::COL_S + CW * g, sv);
+          const unsigned long long c2 = f2(c, c);
+          const bool diag = p.causal && (i == ktile);
+#pragma unroll
+          for (int e = 0; e < CW; e += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse2 + e);
+            float x0, x1, x2, x3;
+            f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
+            f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
+            float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            if (diag) {  // query i*128 + q sees key k0 + r only if q >= r
+              const int q = CW * g + e;
+              if (q < r) p0 = 0.f;
+              if (q + 1 < r) p1 = 0.f;
+              if (q + 2 < r) p2 = 0.f;
+              if (q + 3 < r) p3 = 0.f;
+            }
+            pk[e / 2] = pack_bf16(p0, p1);
+            pk[e / 2 + 1] = pack_bf16(p2, p3);
           }
-          pk[e / 2] = pack_bf16(p0, p1);
-          pk[e / 2 + 1] = pack_bf16(p2, p3);
         }
-      }
-      // P^T over the group's own first CW/2 S^T columns (already read above)
-      tmem_st16(lane_base + C::COL_S + CW * g, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p_ready);
-      FA2_TRACE_AT(trace_row, 8 * g + 2, it);
-      // the previous step's dQ is ready by now (its MMAs ran while P^T was formed)
-      if (it > 0) {
-        ok = drain(it - 1);
+        // P^T over the group's own first CW/2 S^T columns (already read above)
+        tmem_st16(lane_base + C::COL_S + CW * g, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p_ready);
+        FA2_TRACE_AT(trace_row, 8 * g + 2, it);
+        // the previous step's dQ is ready by now (its MMAs ran while P^T was formed)
+        if (it > 0) {
+          ok = drain(it - 1);
+          if (!ok) break;
+        }
+        // dS^T = P^T (dP^T - D) for the same columns, bf16 into the swizzled smem tile
+        ok = mbar_wait(bar_dp_full, gg & 1, abort_flag, 0x1302);
         if (!ok) break;
+        tc_fence_after();
+        uint32_t dk[CW / 2];
+        {
+          float dp[CW];
+          tmem_ld32(lane_base + C::COL_DP + CW * g, dp);
+#pragma unroll
+          for (int e = 0; e < CW; e += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(dlt + e);
+            const unsigned long long pa = f2(__uint_as_float(pk[e / 2] << 16), __uint_as_float(pk[e / 2] & 0xFFFF0000u));
+            const unsigned long long pb = f2(__uint_as_float(pk[e / 2 + 1] << 16), __uint_as_float(pk[e / 2 + 1] & 0xFFFF0000u));
+            const unsigned long long da = f2_add(f2(dp[e], dp[e + 1]), f2(-d4.x, -d4.y));
+            const unsigned long long db = f2_add(f2(dp[e + 2], dp[e + 3]), f2(-d4.z, -d4.w));
+            float s0, s1, s2, s3;
+            f2_split(f2_mul(pa, da), s0, s1);
+            f2_split(f2_mul(pb, db), s2, s3);
+            dk[e / 2] = pack_bf16(s0, s1);
+            dk[e / 2 + 1] = pack_bf16(s2, s3);
+          }
+        }
+        if (gg > 0) {  // dK and dQ of the previous step have finished reading the dS^T tile
+          ok = mbar_wait(bar_dsm_free, (gg - 1) & 1, abort_flag, 0x1303);
+          if (!ok) break;
+        }
+#pragma unroll
+        for (int u = 0; u < CW / 8; ++u) {
+          const uint32_t off = sw128_offset(r, (CW / 8) * g + u);
+          *reinterpret_cast<uint4*>(ds_base + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar_ds_ready);
+        FA2_TRACE_AT(trace_row, 8 * g + 3, it);
       }
-      // dS^T = P^T (dP^T - D) for the same columns, bf16 into the swizzled smem tile
-      ok = mbar_wait(bar_dp_full, it & 1, abort_flag, 0x1302);
+      if (ok) ok = drain(n_iter - 1);
+      if (ok) ok = mbar_wait(bar_dkv_done, n & 1, abort_flag, 0x1305);
+#ifdef FA2_TRACE
+      FA2_TRACE_AT(trace_row, 32, 0);
+#endif
       if (!ok) break;
-      tc_fence_after();
-      uint32_t dk[CW / 2];
+      // epilogue: group g stores d columns [g D/4, (g+1) D/4) of dV and scale * dK;
+      // the TMEM columns are released before the stores
       {
-        float dp[CW];
-        tmem_ld32(lane_base + C::COL_DP + CW * g, dp);
+        constexpr int DW = D / C::NWG;
+        tc_fence_after();
+        const int key = ktile * C::BN + r;
+        const bool store = key < p.N;
+        const size_t off = (static_cast<size_t>(bh) * p.N + key) * D + DW * g;
+        float v[DW], w[DW];
+        if constexpr (DW == 32) {
+          tmem_ld32(lane_base + C::COL_DV + DW * g, v);
+          tmem_ld32(lane_base + C::COL_DK + DW * g, w);
+        } else {
+          tmem_ld16(lane_base + C::COL_DV + DW * g, v);
+          tmem_ld16(lane_base + C::COL_DK + DW * g, w);
+        }
+        tc_fence_before();
+        mbar_arrive(bar_dkv_free);
+        if (store) {
+          uint4 o[DW / 8];
+          uint32_t* ou = reinterpret_cast<uint32_t*>(o);
 #pragma unroll
-        for (int e = 0; e < CW; e += 4) {
-          const float4 d4 = *reinterpret_cast<const float4*>(dlt + e);
-          const unsigned long long pa = f2(__uint_as_float(pk[e / 2] << 16), __uint_as_float(pk[e / 2] & 0xFFFF0000u));
-          const unsigned long long pb = f2(__uint_as_float(pk[e / 2 + 1] << 16), __uint_as_float(pk[e / 2 + 1] & 0xFFFF0000u));
-          const unsigned long long da = f2_add(f2(dp[e], dp[e + 1]), f2(-d4.x, -d4.y));
-          const unsigned long long db = f2_add(f2(dp[e + 2], dp[e + 3]), f2(-d4.z, -d4.w));
-          float s0, s1, s2, s3;
-          f2_split(f2_mul(pa, da), s0, s1);
-          f2_split(f2_mul(pb, db), s2, s3);
-          dk[e / 2] = pack_bf16(s0, s1);
-          dk[e / 2 + 1] = pack_bf16(s2, s3);
+          for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(p.dv + off);
+#pragma unroll
+          for (int e = 0; e < DW / 8; ++e) dst[e] = o[e];
+#pragma unroll
+          for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(w[2 * e] * p.scale, w[2 * e + 1] * p.scale);
+          dst = reinterpret_cast<uint4*>(p.dk + off);
+#pragma unroll
+          for (int e = 0; e < DW / 8; ++e) dst[e] = o[e];
         }
       }
-      if (it > 0) {  // dK_{i-1} and dQ_{i-1} have finished reading the dS^T tile
-        ok = mbar_wait(bar_dsm_free, (it - 1) & 1, abort_flag, 0x1303);
-        if (!ok) break;
-      }
-#pragma unroll
-      for (int u = 0; u < CW / 8; ++u) {
-        const uint32_t off = sw128_offset(r, (CW / 8) * g + u);
-        *reinterpret_cast<uint4*>(ds_base + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-      }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_ds_ready);
-      FA2_TRACE_AT(trace_row, 8 * g + 3, it);
-    }
-    if (ok && n_iter > 0) ok = drain(n_iter - 1);
-    if (ok) ok = mbar_wait(bar_dkv_done, 0, abort_flag, 0x1305);
-    FA2_TRACE_AT(trace_row, 32, 0);
-    if (ok) {
-      // epilogue: group g stores d columns [g D/4, (g+1) D/4) of dV and scale * dK
-      constexpr int DW = D / C::NWG;
-      tc_fence_after();
-      const bool store = key < p.N;
-      const size_t off = (static_cast<size_t>(bh) * p.N + key) * D + DW * g;
-      float v[DW];
-      uint4 w[DW / 8];
-      uint32_t* wu = reinterpret_cast<uint32_t*>(w);
-      if constexpr (DW == 32)
-        tmem_ld32(lane_base + C::COL_DV + DW * g, v);
-      else
-        tmem_ld16(lane_base + C::COL_DV + DW * g, v);
-#pragma unroll
-      for (int e = 0; e < DW / 2; ++e) wu[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-      if (store) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dv + off);
-#pragma unroll
-        for (int e = 0; e < DW / 8; ++e) dst[e] = w[e];
-      }
-      if constexpr (DW == 32)
-        tmem_ld32(lane_base + C::COL_DK + DW * g, v);
-      else
-        tmem_ld16(lane_base + C::COL_DK + DW * g, v);
-#pragma unroll
-      for (int e = 0; e < DW / 2; ++e) wu[e] = pack_bf16(v[2 * e] * p.scale, v[2 * e + 1] * p.scale);
-      if (store) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dk + off);
-#pragma unroll
-        for (int e = 0; e < DW / 8; ++e) dst[e] = w[e];
-      }
+      gs += n_iter;
     }
   }
 

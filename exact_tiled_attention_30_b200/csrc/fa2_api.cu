@@ -89,6 +89,8 @@ fa2_status check_common(int B, int H, int N, int d, float scale) {
   if (!std::isfinite(scale) || scale < 0.f) return FA2_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA2_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > 65535) return FA2_ERR_UNSUPPORTED;
+  // the backward's work items (key tiles x heads) are counted in 32 bits
+  if (static_cast<long long>(B) * H * ((N + 127) / 128) > 0x7FFFFFFFLL) return FA2_ERR_UNSUPPORTED;
   // every tensor index must fit the 32-bit TMA coordinates and our size_t math,
   // and the 128-row tiles a grid dimension (at most 65535)
   if (static_cast<long long>(N) > 65535LL * 128) return FA2_ERR_UNSUPPORTED;
@@ -141,6 +143,7 @@ struct WsLayout {
   float* dq_acc;
   float* delta;
   float* lse2;
+  unsigned int* counter;
   int Np;
 };
 
@@ -150,7 +153,21 @@ WsLayout ws_layout(void* workspace, int BH, int N, int d) {
   w.dq_acc = reinterpret_cast<float*>(workspace);
   w.delta = w.dq_acc + static_cast<size_t>(BH) * w.Np * d;
   w.lse2 = w.delta + static_cast<size_t>(BH) * w.Np;
+  w.counter = reinterpret_cast<unsigned int*>(w.lse2 + static_cast<size_t>(BH) * w.Np);
   return w;
+}
+
+int sm_count(int dev) {
+  static int count[kMaxDevices] = {0};
+  if (count[dev] == 0) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c < 1) {
+      cudaGetLastError();
+      c = 148;
+    }
+    count[dev] = c;
+  }
+  return count[dev];
 }
 
 inline int grid_cap(long long want) {
@@ -168,6 +185,7 @@ fa2_status launch_bwd_pre(const void* o, const float* lse, const void* dO, int B
   pp.dq_acc = w.dq_acc;
   pp.delta = w.delta;
   pp.lse2 = w.lse2;
+  pp.counter = w.counter;
   pp.N = N;
   pp.Np = w.Np;
   pp.rows = static_cast<long long>(BH) * w.Np;
@@ -199,13 +217,18 @@ fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const vo
   bp.dq_acc = w.dq_acc;
   bp.lse2 = w.lse2;
   bp.delta = w.delta;
+  bp.counter = w.counter;
   bp.N = N;
   bp.Np = w.Np;
+  bp.BH = BH;
   bp.n_ktiles = w.Np / 128;
   bp.causal = causal ? 1 : 0;
   bp.scale = scale;
   bp.scale_log2 = scale * 1.4426950408889634f;
-  fa2::fa2_bwd_kernel<D><<<dim3(bp.n_ktiles, BH), C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, bp);
+  // persistent: one CTA per SM (its shared memory allows no second one)
+  const long long items = static_cast<long long>(bp.n_ktiles) * BH;
+  const int ctas = static_cast<int>(items < sm_count(dev) ? items : sm_count(dev));
+  fa2::fa2_bwd_kernel<D><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, bp);
   return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
 
@@ -266,7 +289,7 @@ size_t fa2_backward_workspace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
   const size_t np = (static_cast<size_t>(N) + 127) / 128 * 128;
   const size_t bh = static_cast<size_t>(B) * H;
-  return bh * np * d * 4 + 2 * bh * np * 4;
+  return bh * np * d * 4 + 2 * bh * np * 4 + 16;
 }
 
 fa2_status fa2_backward_preprocess(const void* o, const float* lse, const void* dO, int B, int H,

@@ -71,9 +71,9 @@ FA2_API fa2_status fa2_forward(const void* q, const void* k, const void* v, void
 
 /*
  * Bytes of device workspace fa2_backward needs for these sizes: an fp32 dQ
- * accumulator [B,H,Np,d] plus two fp32 row vectors [B,H,Np] (D = rowsum(dO o O)
- * and the log2-scaled LSE), with Np = N rounded up to 128. Returns 0 for
- * invalid sizes.
+ * accumulator [B,H,Np,d], two fp32 row vectors [B,H,Np] (D = rowsum(dO o O)
+ * and the log2-scaled LSE), with Np = N rounded up to 128, and 16 bytes for the
+ * main kernel's work-item counter. Returns 0 for invalid sizes.
  */
 FA2_API size_t fa2_backward_workspace_size(int B, int H, int N, int d);
 
@@ -98,8 +98,11 @@ FA2_API fa2_status fa2_backward(const void* q, const void* k, const void* v, con
  * arguments and checks as fa2_backward; run them in this order on one stream,
  * with the same workspace, to get exactly fa2_backward's result):
  *  fa2_backward_preprocess  D = rowsum(dO o O), LSE * log2(e), dQ accumulator
- *                           zeroed; padding rows get D = 0 and LSE = +inf.
- *  fa2_backward_main        dK, dV (bf16 outputs) and the fp32 dQ accumulator.
+ *                           and work-item counter zeroed; padding rows get
+ *                           D = 0 and LSE = +inf.
+ *  fa2_backward_main        dK, dV (bf16 outputs) and the fp32 dQ accumulator;
+ *                           one persistent CTA per SM takes (key tile, head)
+ *                           items from the counter.
  *  fa2_backward_dq_convert  dq = bf16(scale * accumulator).
  * Splitting them lets a caller time or overlap the stages individually.
  */

@@ -82,8 +82,8 @@ def test_forward_rejects_bad_arguments(lib):
 def test_workspace_size(lib):
     import exact_tiled_attention_30_b200 as m
 
-    assert m.fa2_backward_workspace_size(1, 1, 128, 64) == 128 * 64 * 4 + 2 * 128 * 4
-    assert m.fa2_backward_workspace_size(2, 3, 129, 128) == 6 * 256 * 128 * 4 + 2 * 6 * 256 * 4
+    assert m.fa2_backward_workspace_size(1, 1, 128, 64) == 128 * 64 * 4 + 2 * 128 * 4 + 16
+    assert m.fa2_backward_workspace_size(2, 3, 129, 128) == 6 * 256 * 128 * 4 + 2 * 6 * 256 * 4 + 16
     assert m.fa2_backward_workspace_size(1, 1, 0, 64) == 0
     assert m.fa2_backward_workspace_size(1, 1, 10, 32) == 0
 
