@@ -45,7 +45,7 @@ WORKLOADS = {
 DEFAULT_WORKLOAD = "fwd_bwd_b8_h16_n2048_d128_causal"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
-    "fa2_fwd_kernel": ["fwd_sm100.cuh", "sm100_ptx.cuh"],
+    "fa2_fwd_kernel": ["fwd_sm100.cuh", "sm100_ptx.cuh", "exp2_poly.cuh"],
     "fa2_bwd_kernel": ["bwd_sm100.cuh", "sm100_ptx.cuh"],
     "fa2_bwd_pre_kernel": ["bwd_sm100.cuh"],
     "fa2_bwd_dq_convert_kernel": ["bwd_sm100.cuh"],
@@ -160,11 +160,28 @@ def flops(w, passes: str, halve_causal: bool = True) -> float:
     return f
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of a list of floats over all ranks (identity on one rank).
+    Every rank must call it with the same number of values."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def rank_config_index(config_index: int, rank: int) -> int:
+    """Seed index of a rank's batch: every rank draws an independent batch."""
+    return config_index + 1000 * rank
+
+
 def make_inputs(w, rank: int):
     import attn_inputs
 
-    return attn_inputs.make_qkvdo(w["cfg"] + 1000 * rank, w["B"], w["H"], w["N"], w["d"],
-                                  with_do=True)
+    return attn_inputs.make_qkvdo(rank_config_index(w["cfg"], rank), w["B"], w["H"], w["N"],
+                                  w["d"], with_do=True)
 
 
 # ------------------------------------------------------------- oracle timing
@@ -354,11 +371,9 @@ def main():
     names = ["fa2_fwd_kernel", "fa2_bwd_pre_kernel", "fa2_bwd_kernel", "fa2_bwd_dq_convert_kernel"]
     kern_ms = {n: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / args.steps
                for j, n in enumerate(names)}
-    if dist:
-        t = torch.tensor([total_ms] + [kern_ms[n] for n in names], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t[0])
-        kern_ms = {n: float(t[1 + j]) for j, n in enumerate(names)}
+    red = max_over_ranks([total_ms] + [kern_ms[n] for n in names], dist, dev)
+    total_ms = red[0]
+    kern_ms = {n: red[1 + j] for j, n in enumerate(names)}
     ms_step = total_ms / args.steps
 
     # e2e through the public API: pinned host inputs in, every output back to host
@@ -382,11 +397,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dist, dev)[0]
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
     d2h = sum(x.numel() * x.element_size() for x in outs_host)
 

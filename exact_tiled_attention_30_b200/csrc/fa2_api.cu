@@ -133,7 +133,8 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   p.n_pairs = (p.n_qtiles + 1) / 2;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const dim3 grid = p.causal ? dim3(BH, p.n_pairs) : dim3(p.n_pairs, BH);
+  p.BH = BH;
+  const dim3 grid = p.causal ? dim3(BH * p.n_pairs) : dim3(p.n_pairs, BH);
   fa2::fa2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
   return FA2_OK;

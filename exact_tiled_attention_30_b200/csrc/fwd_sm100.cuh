@@ -61,6 +61,7 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
   static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 of the largest P entry
+  static constexpr int HEAD_GROUP = 16;                    // causal launch order, see below
   // d = 64: one pair of weights in POLY_EVERY is exponentiated on the FMA pipe
   // (the MUFU unit is the tighter limit there); d = 128: MUFU only (measured faster)
   static constexpr int POLY_EVERY = (D == 64) ? 3 : 1 << 20;
@@ -72,6 +73,7 @@ struct FwdParams {
   int N;
   int n_qtiles;  // ceil(N / 128)
   int n_pairs;   // ceil(n_qtiles / 2)
+  int BH;
   int causal;
   float scale_log2;  // scale * log2(e)
 };
@@ -87,12 +89,22 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Blocks launch in linear order. Causal: grid (batch*head, pair) with the pair
-  // as the slow index, so the heaviest pairs of all heads start first (longest
-  // processing time first). Non-causal: grid (pair, batch*head), so the pairs of
-  // one head run together and share its K/V tiles in L2.
-  const int pair = p.causal ? p.n_pairs - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
-  const int bh = p.causal ? blockIdx.x : blockIdx.y;
+  // Blocks launch in linear order. Non-causal: grid (pair, batch*head), so the
+  // pairs of one head run together and share its K/V tiles in L2. Causal: a 1-D
+  // grid in groups of HEAD_GROUP heads (their K/V stay in L2 while the group
+  // runs); inside a group the heaviest pairs of every head start first.
+  int pair, bh;
+  if (!p.causal) {
+    pair = blockIdx.x;
+    bh = blockIdx.y;
+  } else {
+    const int group_blocks = C::HEAD_GROUP * p.n_pairs;
+    const int grp = static_cast<int>(blockIdx.x) / group_blocks;
+    const int r = static_cast<int>(blockIdx.x) - grp * group_blocks;
+    const int heads = min(C::HEAD_GROUP, p.BH - grp * C::HEAD_GROUP);
+    pair = p.n_pairs - 1 - r / heads;
+    bh = grp * C::HEAD_GROUP + r % heads;
+  }
   const int n_kv_total = (p.N + C::BN - 1) / C::BN;
   // query tiles 2*pair and 2*pair+1; with causal masking tile t sees key tiles [0, qt_t]
   const int qt0 = 2 * pair;
@@ -100,7 +112,7 @@ __global__ void __launch_bounds__(320, 1)
   const int n0 = p.causal ? min(n_kv_total, qt0 + 1) : n_kv_total;
   const int n1 = p.causal ? min(n_kv_total, qt1 + 1) : n_kv_total;  // n1 >= n0
 #ifdef FA2_TRACE
-  const bool trace_cta = blockIdx.y == 0 && blockIdx.x == 7;
+  const bool trace_cta = p.causal ? blockIdx.x == 7 : (blockIdx.x == 0 && blockIdx.y == 7);
 #endif
 
   const uint32_t bar_q = sbase + C::OFF_BAR;

@@ -1,0 +1,97 @@
+"""Host-side pieces of bench.py: FLOP counts, peaks, the ncu traffic record, the
+per-rank seeds and the max-over-ranks timing reduction (world size 2 over gloo)."""
+import json
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_flop_counts():
+    w = dict(B=8, H=16, N=2048, d=128, causal=True)
+    fwd = 4.0 * 8 * 16 * 2048 ** 2 * 128
+    assert bench.flops(w, "fwd") == fwd / 2
+    assert bench.flops(w, "bwd") == 2.5 * fwd / 2
+    assert bench.flops(w, "fwd+bwd") == 3.5 * fwd / 2
+    assert bench.flops(w, "fwd+bwd", halve_causal=False) == 3.5 * fwd
+    assert bench.flops(dict(w, causal=False), "fwd") == fwd
+
+
+def test_default_workload_is_forward_backward():
+    w = bench.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    assert (w["B"], w["H"], w["N"], w["d"], w["causal"]) == (8, 16, 2048, 128, True)
+
+
+def test_peaks_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, kind = bench.load_peaks()
+    assert kind == "fallback" and peaks["bf16_tflops"] == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}))
+    peaks, kind = bench.load_peaks()
+    assert kind == "measured" and peaks["bf16_tflops"] == 1600.0
+
+
+def test_traffic_record_is_dropped_when_the_kernel_changes(tmp_path, monkeypatch):
+    real = bench.kernel_src_hash("fa2_bwd_kernel")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    rec = {"fa2_bwd_kernel": {"dram_bytes_per_launch": 123, "workload": "w", "src_hash": real}}
+    (prof / "ncu_traffic.json").write_text(json.dumps(rec))
+    csrc = os.path.join(bench.ROOT, "exact_tiled_attention_30_b200", "csrc")
+    os.makedirs(tmp_path / "exact_tiled_attention_30_b200")
+    os.symlink(csrc, tmp_path / "exact_tiled_attention_30_b200" / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("fa2_bwd_kernel", "w") == 123
+    assert bench.ncu_traffic("fa2_bwd_kernel", "other workload") is None
+    rec["fa2_bwd_kernel"]["src_hash"] = "0" * 16
+    (prof / "ncu_traffic.json").write_text(json.dumps(rec))
+    assert bench.ncu_traffic("fa2_bwd_kernel", "w") is None
+
+
+def test_ranks_draw_independent_batches():
+    seeds = {bench.rank_config_index(2, r) for r in range(8)}
+    assert len(seeds) == 8
+    w = dict(bench.WORKLOADS[bench.DEFAULT_WORKLOAD], B=1, H=1, N=16, d=64)
+    a, b = bench.make_inputs(w, 0), bench.make_inputs(w, 1)
+    assert not (a["q"] == b["q"]).all()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        got = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 0.5 * rank], dist, "cpu")
+        out[rank] = got
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world_size_2():
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == out[1] == [2.0, 10.0, 0.5]
+
+
+def test_max_over_ranks_single_process():
+    assert bench.max_over_ranks([3, 4.5]) == [3.0, 4.5]
