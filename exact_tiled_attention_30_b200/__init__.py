@@ -18,11 +18,16 @@ import os
 __all__ = [
     "FA2Error", "LIB_PATH", "load_library", "fa2_forward", "fa2_backward", "fa2_backward_workspace_size",
     "fa2_backward_preprocess", "fa2_backward_main", "fa2_backward_dq_convert",
+    "fa2_backward_ex", "fa2_backward_dq_strategy", "fa2_backward_main_dkdv", "fa2_backward_dq",
+    "DQ_AUTO", "DQ_REDUCE", "DQ_SEPARATE",
     "fa2_status_string", "fa2_get_device_status", "fa2_clear_device_status",
     "attention_forward", "attention_backward", "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa2_b200.so")
+
+#: dQ strategies of fa2_backward_ex (fa2_dq_strategy in include/fa2.h)
+DQ_AUTO, DQ_REDUCE, DQ_SEPARATE = 0, 1, 2
 
 STATUS = {0: "FA2_OK", 1: "FA2_ERR_INVALID_ARG", 2: "FA2_ERR_UNSUPPORTED",
           3: "FA2_ERR_MISALIGNED", 4: "FA2_ERR_CUDA", 5: "FA2_ERR_TIMEOUT"}
@@ -62,6 +67,16 @@ def load_library():
     lib.fa2_backward_main.restype = i
     lib.fa2_backward_dq_convert.argtypes = [vp, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t, vp]
     lib.fa2_backward_dq_convert.restype = i
+    lib.fa2_backward_ex.argtypes = [vp] * 9 + [i, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t,
+                                              i, vp]
+    lib.fa2_backward_ex.restype = i
+    lib.fa2_backward_dq_strategy.argtypes = [i, i, i, i, i]
+    lib.fa2_backward_dq_strategy.restype = i
+    lib.fa2_backward_main_dkdv.argtypes = [vp] * 6 + [i, i, i, i, i, ctypes.c_float, vp,
+                                                      ctypes.c_size_t, vp]
+    lib.fa2_backward_main_dkdv.restype = i
+    lib.fa2_backward_dq.argtypes = [vp] * 5 + [i, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t, vp]
+    lib.fa2_backward_dq.restype = i
     lib.fa2_status_string.argtypes = [i]
     lib.fa2_status_string.restype = ctypes.c_char_p
     lib.fa2_get_device_status.argtypes = [vp, ctypes.POINTER(i)]
@@ -175,6 +190,46 @@ def fa2_backward_dq_convert(dq, scale: float, workspace, stream=None) -> None:
         _ptr(dq), B, H, N, d, float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
+def fa2_backward_ex(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float, workspace,
+                    dq_strategy: int = DQ_AUTO, stream=None) -> None:
+    """C ABI fa2_backward_ex: fa2_backward with an explicit dQ strategy."""
+    import torch
+
+    B, H, N, d = _bhnd(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _require(t, n, torch.bfloat16)
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
+    _require(lse, "lse", torch.float32)
+    _require(workspace, "workspace")
+    _check("fa2_backward_ex", load_library().fa2_backward_ex(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, H, N, d, int(bool(causal)), float(scale), _ptr(workspace), _nbytes(workspace),
+        int(dq_strategy), _stream(stream)))
+
+
+def fa2_backward_dq_strategy(B: int, H: int, N: int, d: int, causal: bool) -> int:
+    return int(load_library().fa2_backward_dq_strategy(B, H, N, d, int(bool(causal))))
+
+
+def fa2_backward_main_dkdv(q, k, v, dout, dk, dv, causal: bool, scale: float, workspace,
+                           stream=None) -> None:
+    """C ABI fa2_backward_main_dkdv (dK, dV only; FA2_DQ_SEPARATE)."""
+    B, H, N, d = _bhnd(q)
+    _check("fa2_backward_main_dkdv", load_library().fa2_backward_main_dkdv(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)),
+        float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def fa2_backward_dq(q, k, v, dout, dq, causal: bool, scale: float, workspace, stream=None) -> None:
+    """C ABI fa2_backward_dq (query-parallel dQ kernel; FA2_DQ_SEPARATE)."""
+    B, H, N, d = _bhnd(q)
+    _check("fa2_backward_dq", load_library().fa2_backward_dq(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), B, H, N, d, int(bool(causal)),
+        float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
 def fa2_status_string(status: int) -> str:
     return load_library().fa2_status_string(int(status)).decode()
 
@@ -204,8 +259,8 @@ def attention_forward(q, k, v, causal: bool = False, scale: float | None = None,
 
 
 def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
-                       stream=None, workspace=None):
-    """Allocates dq, dk, dv (and the workspace unless given), runs fa2_backward."""
+                       stream=None, workspace=None, dq_strategy: int = DQ_AUTO):
+    """Allocates dq, dk, dv (and the workspace unless given), runs fa2_backward_ex."""
     import torch
 
     B, H, N, d = _bhnd(q)
@@ -215,7 +270,7 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: float
     if workspace is None:
         workspace = torch.empty(fa2_backward_workspace_size(B, H, N, d), dtype=torch.uint8,
                                 device=q.device)
-    fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, stream)
+    fa2_backward_ex(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, dq_strategy, stream)
     return dq, dk, dv
 
 

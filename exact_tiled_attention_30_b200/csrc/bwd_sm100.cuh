@@ -237,7 +237,9 @@ __device__ __forceinline__ void decode_item(int item, int n_ktiles, int BH, int 
   bh = grp * head_group + (r - ktile * heads);
 }
 
-template <int D>
+// WITH_DQ = false is the dK/dV-only variant used when dQ comes from the
+// separate query-parallel kernel (fa2_bwd_dq_kernel).
+template <int D, bool WITH_DQ>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -432,7 +434,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           const int s = g % C::STAGES;
           const uint32_t acc0 = it > 0 ? 1u : 0u;
           FA2_TRACE_AT(trace_cta && n == 0, 16, it);
-          if (C::DQ_IN_DP && g > 0) {  // the dP^T columns hold dQ of step g-1 until read out
+          if (WITH_DQ && C::DQ_IN_DP && g > 0) {  // the dP^T columns hold dQ of step g-1 until read out
             ok = mbar_wait(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1203);
             if (!ok) break;
             tc_fence_after();
@@ -478,21 +480,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           for (int k = 0; k < C::BM / 16; ++k)
             umma_ss2(tmem + C::COL_DK, dSk.lo + kmaj(k), dSk.hi, qmlo + k * (2048 >> 4), dQm.hi,
                      IDESC_KV, k > 0 ? 1u : acc0);
-          if (!C::DQ_IN_DP && g > 0) {  // dQ of step g-1 must be read out before it is overwritten
-            ok = mbar_wait(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1206);
-            if (!ok) break;
-            tc_fence_after();
+          if constexpr (WITH_DQ) {
+            if (!C::DQ_IN_DP && g > 0) {  // dQ of step g-1 must be read out before it is overwritten
+              ok = mbar_wait(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1206);
+              if (!ok) break;
+              tc_fence_after();
+            }
+  #pragma unroll
+            for (int k = 0; k < C::BN / 16; ++k) {  // reduction over the 128 keys
+              if (C::DQ_T)  // dQ^T = K^T dS^T
+                umma_ss2(tmem + C::COL_DQ, dKm.lo + k * (2048 >> 4), dKm.hi, dSm.lo + k * (2048 >> 4),
+                         dSm.hi, IDESC_QT, k > 0 ? 1u : 0u);
+              else  // dQ = dS K
+                umma_ss2(tmem + C::COL_DQ, dSm.lo + k * (2048 >> 4), dSm.hi, dKm.lo + k * (2048 >> 4),
+                         dKm.hi, IDESC_Q, k > 0 ? 1u : 0u);
+            }
+            umma_commit(bar_dq_full);
           }
-#pragma unroll
-          for (int k = 0; k < C::BN / 16; ++k) {  // reduction over the 128 keys
-            if (C::DQ_T)  // dQ^T = K^T dS^T
-              umma_ss2(tmem + C::COL_DQ, dKm.lo + k * (2048 >> 4), dKm.hi, dSm.lo + k * (2048 >> 4),
-                       dSm.hi, IDESC_QT, k > 0 ? 1u : 0u);
-            else  // dQ = dS K
-              umma_ss2(tmem + C::COL_DQ, dSm.lo + k * (2048 >> 4), dSm.hi, dKm.lo + k * (2048 >> 4),
-                       dKm.hi, IDESC_Q, k > 0 ? 1u : 0u);
-          }
-          umma_commit(bar_dq_full);
           umma_commit(bar_dsm_free);
           umma_commit(bar_st_empty(s));
         }
@@ -604,7 +608,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         mbar_arrive(bar_p_ready);
         FA2_TRACE_AT(trace_row, 8 * g + 2, it);
         // the previous step's dQ is ready by now (its MMAs ran while P^T was formed)
-        if (it > 0) {
+        if (WITH_DQ && it > 0) {
           ok = drain(it - 1);
           if (!ok) break;
         }
@@ -644,7 +648,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         mbar_arrive(bar_ds_ready);
         FA2_TRACE_AT(trace_row, 8 * g + 3, it);
       }
-      if (ok) ok = drain(n_iter - 1);
+      if (WITH_DQ && ok) ok = drain(n_iter - 1);
       if (ok) ok = mbar_wait(bar_dkv_done, n & 1, abort_flag, 0x1305);
 #ifdef FA2_TRACE
       FA2_TRACE_AT(trace_row, 32, 0);
@@ -691,6 +695,304 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 33, 0);
+  if (warp == C::WARP_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------ dQ kernel (B3b)
+// dQ by a separate, query-parallel kernel: one CTA per (128-row query block i,
+// batch*head) loops over the key blocks j (causal: j <= i) and recomputes
+//   S = Q_i K_j^T,  P = exp2(c S - LSE2),  dP = dO_i V_j^T,  dS = P (dP - D),
+//   dQ_i += dS K_j   (accumulated in TMEM; scaled and stored once, no atomics).
+// Queries sit on TMEM lanes, so LSE2 and D are one register per thread.
+//   warp 16       TMA producer: Q_i, dO_i once, then K_j/V_j into a 2-stage ring
+//   warp 17       MMA issuer: S_j, dP_j; after dS_j is in smem, S_{j+1}, dP_{j+1}
+//                 and then dQ += dS_j K_j (so the next elementwise pass overlaps it)
+//   warps 0-15    four elementwise warpgroups, group g owns keys [32g, 32g+32)
+// Tensor memory: S [0,128), dP [128,256), dQ [256,256+D).
+template <int D>
+struct BwdDqCfg {
+  static constexpr int BM = 128, BN = 128, STAGES = 2;
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int CHUNK_BYTES = 128 * 128;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = TILE_BYTES;
+  static constexpr int OFF_K = 2 * TILE_BYTES;                  // + s * 2 * TILE_BYTES
+  static constexpr int OFF_V = 3 * TILE_BYTES;                  // + s * 2 * TILE_BYTES
+  static constexpr int OFF_DS = TILE_BYTES * (2 + 2 * STAGES);  // 128 x 128 bf16, [query][key]
+  static constexpr int OFF_BAR = OFF_DS + 32768;
+  // q_full, kv_full[S], kv_empty[S], s_full, dp_full, ds_ready, dsm_free, dq_done, drain
+  static constexpr int NUM_BARS = 1 + 2 * STAGES + 6;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+  static constexpr int NWG = 4, CW = 128 / NWG;
+  static constexpr int WARP_TMA = 4 * NWG, WARP_MMA = 4 * NWG + 1;
+  static constexpr int THREADS = 32 * (4 * NWG + 2);
+  static constexpr int ELEM_THREADS = 128 * NWG;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256;
+  static constexpr int HEAD_GROUP = 16;
+};
+
+struct BwdDqParams {
+  __nv_bfloat16* dq;
+  const float* lse2;   // [BH][Np]
+  const float* delta;  // [BH][Np]
+  int N;
+  int Np;
+  int BH;
+  int n_qtiles;
+  int causal;
+  float scale;
+  float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(BwdDqCfg<D>::THREADS, 1)
+    fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                      const BwdDqParams p) {
+  using C = BwdDqCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Non-causal: grid (query tile, batch*head). Causal: 1-D grid in groups of
+  // HEAD_GROUP heads with the query tiles that see the most key tiles first.
+  int qtile, bh;
+  if (!p.causal) {
+    qtile = blockIdx.x;
+    bh = blockIdx.y;
+  } else {
+    const int group_blocks = C::HEAD_GROUP * p.n_qtiles;
+    const int grp = static_cast<int>(blockIdx.x) / group_blocks;
+    const int r = static_cast<int>(blockIdx.x) - grp * group_blocks;
+    const int heads = min(C::HEAD_GROUP, p.BH - grp * C::HEAD_GROUP);
+    qtile = p.n_qtiles - 1 - r / heads;
+    bh = grp * C::HEAD_GROUP + r % heads;
+  }
+  const int n_kv = p.causal ? qtile + 1 : p.n_qtiles;  // self-attention: key tiles = query tiles
+
+  const uint32_t bar_q = sbase + C::OFF_BAR;
+  auto bar_kv_full = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + s); };
+  auto bar_kv_empty = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + C::STAGES + s); };
+  const uint32_t bar_s_full = sbase + C::OFF_BAR + 8 * (1 + 2 * C::STAGES);
+  const uint32_t bar_dp_full = bar_s_full + 8;
+  const uint32_t bar_ds_ready = bar_s_full + 16;
+  const uint32_t bar_dsm_free = bar_s_full + 24;
+  const uint32_t bar_dq_done = bar_s_full + 32;
+  const uint32_t bar_drain = bar_s_full + 40;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar_kv_full(s), 1);
+      mbar_init(bar_kv_empty(s), 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_ds_ready, C::ELEM_THREADS);
+    mbar_init(bar_dsm_free, 1);
+    mbar_init(bar_dq_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::WARP_TMA && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::WARP_TMA) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+      for (int c = 0; c < C::CHUNKS; ++c) {
+        tma_load_3d(sbase + C::OFF_Q + c * C::CHUNK_BYTES, &tm_q, bar_q, c * 64, qtile * C::BM, bh);
+        tma_load_3d(sbase + C::OFF_DO + c * C::CHUNK_BYTES, &tm_do, bar_q, c * 64, qtile * C::BM, bh);
+      }
+      int last_parity[C::STAGES];
+      for (int s = 0; s < C::STAGES; ++s) last_parity[s] = -1;
+      bool ok = true;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int s = j % C::STAGES;
+        const int n = j / C::STAGES;
+        if (n > 0) ok = mbar_wait(bar_kv_empty(s), (n - 1) & 1, abort_flag, 0x1401);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_kv_full(s), 2 * C::TILE_BYTES);
+        for (int c = 0; c < C::CHUNKS; ++c) {
+          tma_load_3d(sbase + C::OFF_K + s * 2 * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_k,
+                      bar_kv_full(s), c * 64, j * C::BN, bh);
+          tma_load_3d(sbase + C::OFF_V + s * 2 * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_v,
+                      bar_kv_full(s), c * 64, j * C::BN, bh);
+        }
+        last_parity[s] = n & 1;
+      }
+      mbar_wait(bar_q, 0, abort_flag, 0x1402);
+      for (int s = 0; s < C::STAGES; ++s)
+        if (last_parity[s] >= 0) mbar_wait(bar_kv_full(s), last_parity[s], abort_flag, 0x1403);
+    }
+  } else if (warp == C::WARP_MMA) {
+    // --------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_SS = idesc_bf16(128, 128, false, false);  // S, dP
+      constexpr uint32_t IDESC_DQ = idesc_bf16(128, D, false, true);     // dQ += dS K
+      const SDesc dQk = sdesc_make(sbase + C::OFF_Q, 16, 1024);
+      const SDesc dOk = sdesc_make(sbase + C::OFF_DO, 16, 1024);
+      const SDesc dK = sdesc_make(sbase + C::OFF_K, 16, 1024);
+      const SDesc dV = sdesc_make(sbase + C::OFF_V, 16, 1024);
+      const SDesc dKm = sdesc_make(sbase + C::OFF_K, C::CHUNK_BYTES, 1024);
+      const SDesc dSk = sdesc_make(sbase + C::OFF_DS, 16, 1024);
+      constexpr uint32_t STAGE16 = 2 * C::TILE_BYTES / 16;
+      auto kmaj = [](int k) -> uint32_t { return ((k >> 2) * C::CHUNK_BYTES + (k & 3) * 32) >> 4; };
+      auto issue_s_dp = [&](int j) {  // S = Q K_j^T, dP = dO V_j^T
+        const uint32_t klo = dK.lo + (j % C::STAGES) * STAGE16;
+        const uint32_t vlo = dV.lo + (j % C::STAGES) * STAGE16;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          umma_ss2(tmem + C::COL_S, dQk.lo + kmaj(k), dQk.hi, klo + kmaj(k), dK.hi, IDESC_SS,
+                   k > 0 ? 1u : 0u);
+        umma_commit(bar_s_full);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          umma_ss2(tmem + C::COL_DP, dOk.lo + kmaj(k), dOk.hi, vlo + kmaj(k), dV.hi, IDESC_SS,
+                   k > 0 ? 1u : 0u);
+        umma_commit(bar_dp_full);
+      };
+      bool ok = mbar_wait(bar_q, 0, abort_flag, 0x1501) &&
+                mbar_wait(bar_kv_full(0), 0, abort_flag, 0x1502);
+      if (ok) {
+        tc_fence_after();
+        issue_s_dp(0);
+      }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        // the elementwise warps have read S_j and dP_j and written dS_j
+        ok = mbar_wait(bar_ds_ready, j & 1, abort_flag, 0x1503);
+        if (!ok) break;
+        tc_fence_after();
+        if (j + 1 < n_kv) {
+          ok = mbar_wait(bar_kv_full((j + 1) % C::STAGES), ((j + 1) / C::STAGES) & 1, abort_flag, 0x1504);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s_dp(j + 1);
+        }
+        const uint32_t kmlo = dKm.lo + (j % C::STAGES) * STAGE16;
+#pragma unroll
+        for (int k = 0; k < C::BN / 16; ++k)  // dQ += dS_j K_j (reduction over keys)
+          umma_ss2(tmem + C::COL_DQ, dSk.lo + kmaj(k), dSk.hi, kmlo + k * (2048 >> 4), dKm.hi,
+                   IDESC_DQ, (j > 0 || k > 0) ? 1u : 0u);
+        umma_commit(bar_dsm_free);
+        umma_commit(bar_kv_empty(j % C::STAGES));
+      }
+      umma_commit(bar_dq_done);
+      umma_commit(bar_drain);
+      mbar_wait(bar_drain, 0, abort_flag, 0x1505);
+    }
+  } else {
+    // ------------------------------------------------ elementwise groups (0-15)
+    constexpr int CW = C::CW;
+    const int g = warp >> 2;           // key-column group
+    const int r = threadIdx.x & 127;   // TMEM lane: query row
+    const int qrow = qtile * C::BM + r;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const size_t vrow = static_cast<size_t>(bh) * p.Np + qrow;
+    const float lse2 = p.lse2[vrow];   // +inf on padding rows: P = 0 there
+    const float dlt = p.delta[vrow];
+    const unsigned long long c2 = f2(p.scale_log2, p.scale_log2);
+    const unsigned long long nl2 = f2(-lse2, -lse2);
+    const unsigned long long nd2 = f2(-dlt, -dlt);
+    uint8_t* ds_base = smem + C::OFF_DS;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      ok = mbar_wait(bar_s_full, j & 1, abort_flag, 0x1601);
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = p.causal && j == qtile;
+      uint32_t pk[CW / 2];
+      {
+        float sv[CW];
+        tmem_ld32(lane_base + C::COL_S + CW * g, sv);
+#pragma unroll
+        for (int e = 0; e < CW; e += 2) {
+          float x0, x1;
+          f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, nl2), x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
+          if (diag) {  // key j*128 + k is visible to query row r only if k <= r
+            const int kk = CW * g + e;
+            if (kk > r) p0 = 0.f;
+            if (kk + 1 > r) p1 = 0.f;
+          }
+          pk[e / 2] = pack_bf16(p0, p1);
+        }
+      }
+      ok = mbar_wait(bar_dp_full, j & 1, abort_flag, 0x1602);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dk[CW / 2];
+      {
+        float dp[CW];
+        tmem_ld32(lane_base + C::COL_DP + CW * g, dp);
+#pragma unroll
+        for (int e = 0; e < CW; e += 2) {
+          const unsigned long long pp = f2(__uint_as_float(pk[e / 2] << 16), __uint_as_float(pk[e / 2] & 0xFFFF0000u));
+          float s0, s1;
+          f2_split(f2_mul(pp, f2_add(f2(dp[e], dp[e + 1]), nd2)), s0, s1);
+          dk[e / 2] = pack_bf16(s0, s1);
+        }
+      }
+      if (j > 0) {  // dQ += dS_{j-1} K_{j-1} has finished reading the dS tile
+        ok = mbar_wait(bar_dsm_free, (j - 1) & 1, abort_flag, 0x1603);
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int u = 0; u < CW / 8; ++u) {
+        const uint32_t off = sw128_offset(r, (CW / 8) * g + u);
+        *reinterpret_cast<uint4*>(ds_base + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_ds_ready);
+    }
+    if (ok) ok = mbar_wait(bar_dq_done, 0, abort_flag, 0x1604);
+    if (ok) {
+      // group g stores d columns [g D/4, (g+1) D/4) of scale * dQ (the TMEM load
+      // is warp-collective, so padding rows load too and only skip the store)
+      constexpr int DW = D / C::NWG;
+      tc_fence_after();
+      float v[DW];
+      if constexpr (DW == 32)
+        tmem_ld32(lane_base + C::COL_DQ + DW * g, v);
+      else
+        tmem_ld16(lane_base + C::COL_DQ + DW * g, v);
+      if (qrow < p.N) {
+        uint4 o[DW / 8];
+        uint32_t* ou = reinterpret_cast<uint32_t*>(o);
+#pragma unroll
+        for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(v[2 * e] * p.scale, v[2 * e + 1] * p.scale);
+        uint4* dst = reinterpret_cast<uint4*>(p.dq + (static_cast<size_t>(bh) * p.N + qrow) * D + DW * g);
+#pragma unroll
+        for (int e = 0; e < DW / 8; ++e) dst[e] = o[e];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   if (warp == C::WARP_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 

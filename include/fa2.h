@@ -94,6 +94,33 @@ FA2_API fa2_status fa2_backward(const void* q, const void* k, const void* v, con
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * How the backward produces dQ (the pages' two options; the default is chosen
+ * by measurement, see fa2_backward_dq_strategy):
+ *  FA2_DQ_REDUCE    the key-block kernel adds each step's dQ into an fp32
+ *                   accumulator in the workspace with reductions; a third
+ *                   kernel converts it to bf16.
+ *  FA2_DQ_SEPARATE  the key-block kernel computes dK, dV only; a separate
+ *                   query-parallel kernel recomputes S, P, dP, dS per query
+ *                   block and accumulates dQ on chip (no atomics, bitwise
+ *                   reproducible dQ, 40% more tensor work).
+ */
+typedef enum { FA2_DQ_AUTO = 0, FA2_DQ_REDUCE = 1, FA2_DQ_SEPARATE = 2 } fa2_dq_strategy;
+
+/* The strategy FA2_DQ_AUTO uses for these sizes (FA2_DQ_REDUCE or FA2_DQ_SEPARATE). */
+FA2_API int fa2_backward_dq_strategy(int B, int H, int N, int d, int causal);
+
+/*
+ * fa2_backward with an explicit dQ strategy (FA2_DQ_*; anything else is
+ * FA2_ERR_INVALID_ARG). Same arguments, workspace and results otherwise.
+ * fa2_backward(...) is fa2_backward_ex(..., FA2_DQ_AUTO, stream).
+ */
+FA2_API fa2_status fa2_backward_ex(const void* q, const void* k, const void* v, const void* o,
+                                   const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                   int B, int H, int N, int d, int causal, float scale,
+                                   void* workspace, size_t workspace_bytes, int dq_strategy,
+                                   void* stream);
+
+/*
  * The three stages fa2_backward launches, callable one at a time (same
  * arguments and checks as fa2_backward; run them in this order on one stream,
  * with the same workspace, to get exactly fa2_backward's result):
@@ -115,6 +142,19 @@ FA2_API fa2_status fa2_backward_main(const void* q, const void* k, const void* v
                                      void* stream);
 FA2_API fa2_status fa2_backward_dq_convert(void* dq, int B, int H, int N, int d, float scale,
                                            void* workspace, size_t workspace_bytes, void* stream);
+/*
+ * The FA2_DQ_SEPARATE stages, after fa2_backward_preprocess:
+ *  fa2_backward_main_dkdv   dK, dV only (the key-block kernel without dQ).
+ *  fa2_backward_dq          dq = scale * dS K by the query-parallel kernel
+ *                           (reads D and LSE from the workspace).
+ */
+FA2_API fa2_status fa2_backward_main_dkdv(const void* q, const void* k, const void* v,
+                                          const void* dO, void* dk, void* dv, int B, int H, int N,
+                                          int d, int causal, float scale, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+FA2_API fa2_status fa2_backward_dq(const void* q, const void* k, const void* v, const void* dO,
+                                   void* dq, int B, int H, int N, int d, int causal, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Backward pass that allocates nothing and takes no workspace. (The paper has

@@ -125,3 +125,13 @@ def test_backward_stages_reject_bad_arguments(lib):
     assert lib.fa2_backward_dq_convert(None, 1, 1, 128, 64, f(0.1), A, ws, None) == 1
     assert lib.fa2_backward_dq_convert(A, 1, 1, 128, 64, f(0.1), A, 16, None) == 1
     assert lib.fa2_backward_dq_convert(A + 2, 1, 1, 128, 64, f(0.1), A, ws, None) == 3
+
+
+def test_backward_ex_rejects_bad_strategy(lib):
+    ws = lib.fa2_backward_workspace_size(1, 1, 128, 64)
+    args = [A] * 9 + [1, 1, 128, 64, 0, ctypes.c_float(0.125), A, ws]
+    assert lib.fa2_backward_ex(*args, 3, None) == 1
+    assert lib.fa2_backward_ex(*args, -1, None) == 1
+    assert lib.fa2_backward_dq_strategy(1, 1, 128, 64, 0) in (1, 2)
+    assert lib.fa2_backward_dq(None, A, A, A, A, 1, 1, 128, 64, 0, ctypes.c_float(0.1), A, ws, None) == 1
+    assert lib.fa2_backward_main_dkdv(A, A, A, A, A, A, 1, 1, 128, 64, 0, ctypes.c_float(0.1), A, 8, None) == 1

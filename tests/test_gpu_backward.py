@@ -30,10 +30,14 @@ def fa2():
     return m
 
 
-def run_fwd_bwd(fa2, t, causal, scale):
+STRATEGIES = pytest.mark.parametrize("strategy", [1, 2], ids=["reduce", "separate"])
+
+
+def run_fwd_bwd(fa2, t, causal, scale, strategy=0):
     q, k, v, do = (gh.to_device(t[n]) for n in ("q", "k", "v", "do"))
     o, lse = fa2.attention_forward(q, k, v, causal=causal, scale=scale)
-    dq, dk, dv = fa2.attention_backward(q, k, v, o, lse, do, causal=causal, scale=scale)
+    dq, dk, dv = fa2.attention_backward(q, k, v, o, lse, do, causal=causal, scale=scale,
+                                        dq_strategy=strategy)
     st, site = fa2.fa2_get_device_status()
     assert st == 0, f"device status {fa2.fa2_status_string(st)} at site {site:#x}"
     return {"dq": gh.to_host_f64(dq), "dk": gh.to_host_f64(dk), "dv": gh.to_host_f64(dv),
@@ -64,11 +68,12 @@ SMALL = [
 ]
 
 
+@STRATEGIES
 @pytest.mark.parametrize("cfg,B,H,N,d,causal", SMALL)
-def test_backward_small(fa2, oracle_mod, cfg, B, H, N, d, causal):
+def test_backward_small(fa2, oracle_mod, cfg, B, H, N, d, causal, strategy):
     t = gh.inputs(cfg, B, H, N, d, with_do=True)
     scale = 1.0 / math.sqrt(d)
-    got = run_fwd_bwd(fa2, t, causal, scale)
+    got = run_fwd_bwd(fa2, t, causal, scale, strategy)
     ref = oracle_mod.attention_backward(t["q"], t["k"], t["v"], t["do"], causal, scale)
     check_grads(got, ref)
     # per-head too, so that one wrong head cannot hide in the global norm
@@ -78,18 +83,20 @@ def test_backward_small(fa2, oracle_mod, cfg, B, H, N, d, causal):
                         {n: ref[n][b, h] for n in ("dq", "dk", "dv")}, f"head ({b},{h})")
 
 
+@STRATEGIES
 @pytest.mark.parametrize("d", [64, 128])
-def test_backward_single_token(fa2, d):
+def test_backward_single_token(fa2, d, strategy):
     """N = 1: dV = dO exactly, dQ = dK = 0 up to rounding."""
     t = gh.inputs(11, 2, 2, 1, d, with_do=True)
-    got = run_fwd_bwd(fa2, t, True, 1.0 / math.sqrt(d))
+    got = run_fwd_bwd(fa2, t, True, 1.0 / math.sqrt(d), strategy)
     np.testing.assert_array_equal(got["dv"], gh.to_host_f64(gh.to_device(t["do"])))
     assert np.abs(got["dq"]).max() <= 1e-3 and np.abs(got["dk"]).max() <= 1e-3
 
 
-def test_backward_scale_zero(fa2, oracle_mod):
+@STRATEGIES
+def test_backward_scale_zero(fa2, oracle_mod, strategy):
     t = gh.inputs(17, 1, 2, 200, 64, with_do=True)
-    got = run_fwd_bwd(fa2, t, True, 0.0)
+    got = run_fwd_bwd(fa2, t, True, 0.0, strategy)
     ref = oracle_mod.attention_backward(t["q"], t["k"], t["v"], t["do"], True, 0.0)
     for name in ("dk", "dv"):
         assert np.isfinite(got[name]).all()
@@ -121,11 +128,12 @@ LARGE_FULL_HEADS = [
 ]
 
 
+@STRATEGIES
 @pytest.mark.parametrize("cfg,B,H,N,d,causal", LARGE_FULL_HEADS)
-def test_backward_large_heads(fa2, oracle_mod, cfg, B, H, N, d, causal):
+def test_backward_large_heads(fa2, oracle_mod, cfg, B, H, N, d, causal, strategy):
     t = gh.inputs(cfg, B, H, N, d, with_do=True)
     scale = 1.0 / math.sqrt(d)
-    got = run_fwd_bwd(fa2, t, causal, scale)
+    got = run_fwd_bwd(fa2, t, causal, scale, strategy)
     for b, h in gh.sample_heads(B, H, 2, seed=cfg):
         ref = oracle_mod.attention_backward(t["q"][b, h], t["k"][b, h], t["v"][b, h],
                                             t["do"][b, h], causal, scale)
@@ -140,11 +148,12 @@ LONG_ROWS = [
 ]
 
 
+@STRATEGIES
 @pytest.mark.parametrize("cfg,B,H,N,d,causal", LONG_ROWS)
-def test_backward_long_sampled_rows(fa2, oracle_mod, cfg, B, H, N, d, causal):
+def test_backward_long_sampled_rows(fa2, oracle_mod, cfg, B, H, N, d, causal, strategy):
     t = gh.inputs(cfg, B, H, N, d, with_do=True)
     scale = 1.0 / math.sqrt(d)
-    got = run_fwd_bwd(fa2, t, causal, scale)
+    got = run_fwd_bwd(fa2, t, causal, scale, strategy)
     rows = gh.sample_rows(N, 48, seed=cfg)
     (b, h), = gh.sample_heads(B, H, 1, seed=cfg)[-1:]
     dq, dk, dv = oracle_mod.attention_backward_rows(t["q"][b, h], t["k"][b, h], t["v"][b, h],
@@ -152,3 +161,30 @@ def test_backward_long_sampled_rows(fa2, oracle_mod, cfg, B, H, N, d, causal):
     check_grads({"dq": got["dq"][b, h, rows], "dk": got["dk"][b, h, rows],
                  "dv": got["dv"][b, h, rows]}, {"dq": dq, "dk": dk, "dv": dv},
                 f"head ({b},{h}) sampled rows")
+
+
+def test_separate_dq_is_bitwise_repeatable(fa2):
+    """The query-parallel dQ kernel has no atomics: repeated runs give identical dQ."""
+    import torch
+
+    t = gh.inputs(22, 2, 4, 640, 128, with_do=True)
+    q, k, v, do = (gh.to_device(t[n]) for n in ("q", "k", "v", "do"))
+    o, lse = fa2.attention_forward(q, k, v, causal=True)
+    ref = fa2.attention_backward(q, k, v, o, lse, do, causal=True, dq_strategy=fa2.DQ_SEPARATE)
+    for _ in range(5):
+        got = fa2.attention_backward(q, k, v, o, lse, do, causal=True, dq_strategy=fa2.DQ_SEPARATE)
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)
+
+
+def test_strategies_agree(fa2):
+    """Both dQ strategies produce the same dK, dV bits and dQ within rounding."""
+    t = gh.inputs(23, 1, 4, 768, 64, with_do=True)
+    q, k, v, do = (gh.to_device(t[n]) for n in ("q", "k", "v", "do"))
+    o, lse = fa2.attention_forward(q, k, v, causal=False)
+    a = fa2.attention_backward(q, k, v, o, lse, do, dq_strategy=fa2.DQ_REDUCE)
+    b = fa2.attention_backward(q, k, v, o, lse, do, dq_strategy=fa2.DQ_SEPARATE)
+    import torch
+
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert gh.rel_fro(gh.to_host_f64(a[0]), gh.to_host_f64(b[0])) < 5e-3
