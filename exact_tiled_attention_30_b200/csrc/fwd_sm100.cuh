@@ -12,15 +12,22 @@
 //     the diagonal tile of each query tile is masked elementwise.
 //
 // B200 mapping (the pages' A100/H100 tiling is prior art only):
-//   warp 8        TMA producer: Q0, Q1 once, then K_j/V_j into a STAGES-deep ring
-//   warp 9        MMA issuer + TMEM owner. Per key tile j it issues
+//   warp 16       TMA producer: Q0, Q1 once, then K_j/V_j into a STAGES-deep ring
+//   warp 17       MMA issuer + TMEM owner. Per key tile j it issues
 //                 PV0_j, S0_{j+1}, PV1_j, S1_{j+1} (in that order), so while one
-//                 warpgroup runs the softmax of its tile the tensor core works on
-//                 the other tile: S_t = Q_t K_j^T (smem x smem -> TMEM) and
-//                 O_t += P_t V_j (P from TMEM, V from smem).
-//   warps 0-3     softmax of query tile 0, warps 4-7 of query tile 1: thread r
-//                 owns row r (TMEM lane r); tcgen05.ld of S, row max, exp2,
-//                 row sum, P written back as bf16 over the first 64 columns of S.
+//                 tile's softmax runs the tensor core works on the other tile:
+//                 S_t = Q_t K_j^T (smem x smem -> TMEM) and O_t += P_t V_j (P from
+//                 TMEM, V from smem). The single issue order also keeps the two
+//                 tiles' softmax phases apart (measured: one issuer per tile let
+//                 them drift into step and contend for the MUFU unit).
+//   warps 0-7     softmax of query tile 0, warps 8-15 of query tile 1. Two
+//                 warpgroups per tile split each row: warpgroup h owns keys
+//                 [64h, 64h+64) of row r (TMEM lane r): tcgen05.ld of its 64
+//                 scores, partial row max (exchanged with the other half through
+//                 shared memory, so both use one reference max), exp2, partial
+//                 row sums, P written back as bf16 over the first 32 of its S
+//                 columns. Halving the per-thread row shortens the softmax step
+//                 that sits between the two MMAs of a tile.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D). Scores are kept in base 2: c = scale * log2(e) folds the
 // softmax scale into the exponent and m is stored pre-multiplied by c.
@@ -52,12 +59,18 @@ struct FwdCfg {
   static constexpr int OFF_K = 2 * TILE_BYTES;        // + s * 2 * TILE_BYTES
   static constexpr int OFF_V = 3 * TILE_BYTES;        // + s * 2 * TILE_BYTES
   static constexpr int OFF_BAR = TILE_BYTES * (2 + 2 * STAGES);
-  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
-  static constexpr int NUM_BARS = 1 + 2 * STAGES + 7;
+  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain,
+  // xmax[2 tiles][2 slots], xsum[2 tiles]
+  static constexpr int NUM_BARS = 1 + 2 * STAGES + 7 + 6;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;  // tmem slot, abort flag
-  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  // exchange between the two halves of a row: partial maxima [tile][slot][half][row]
+  // and, at the end, partial sums [tile][half][l | lr][row]
+  static constexpr int OFF_XMAX = OFF_MISC + 16;
+  static constexpr int OFF_XSUM = OFF_XMAX + 2 * 2 * 2 * 128 * 4;
+  static constexpr int SMEM_BYTES = OFF_XSUM + 2 * 2 * 2 * 128 * 4;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;     // slack for 1024-byte alignment
-  static constexpr int THREADS = 320;
+  static constexpr int WARP_TMA = 16, WARP_MMA = 17;
+  static constexpr int THREADS = 32 * 18;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
   static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 of the largest P entry
@@ -79,7 +92,7 @@ struct FwdParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = FwdCfg<D>;
@@ -123,6 +136,8 @@ __global__ void __launch_bounds__(320, 1)
   auto bar_p_full = [&](int t) { return bar_base + 16 + 8 * t; };
   auto bar_o_done = [&](int t) { return bar_base + 32 + 8 * t; };
   const uint32_t bar_drain = bar_base + 48;
+  auto bar_xmax = [&](int t, int slot) { return bar_base + 56 + 16 * t + 8 * slot; };
+  auto bar_xsum = [&](int t) { return bar_base + 88 + 8 * t; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -134,18 +149,21 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s_full(t), 1);
-      mbar_init(bar_p_full(t), 128);
+      mbar_init(bar_p_full(t), 256);
       mbar_init(bar_o_done(t), 1);
+      mbar_init(bar_xmax(t, 0), 256);
+      mbar_init(bar_xmax(t, 1), 256);
+      mbar_init(bar_xsum(t), 256);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == C::WARP_TMA && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
@@ -155,7 +173,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == C::WARP_TMA) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
@@ -186,7 +204,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int s = 0; s < C::STAGES; ++s)
         if (last_parity[s] >= 0) mbar_wait(bar_kv_full(s), last_parity[s], abort_flag, 0x103);
     }
-  } else if (warp == 9) {
+  } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(128, C::BN, false, false);
@@ -215,8 +233,10 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k) {
-          // V: MN-major (d contiguous), 16 keys = 2 swizzle atoms of 8 rows
-          umma_ts2(ocol, pcol + k * 8, vlo + k * (2048 >> 4), dv0.hi, IDESC_O, k > 0 ? 1u : acc0);
+          // V: MN-major (d contiguous), 16 keys = 2 swizzle atoms of 8 rows. P of
+          // keys [64h, 64h+64) sits in columns [64h, 64h+32)
+          umma_ts2(ocol, pcol + k * 8 + (k >= 4 ? 32 : 0), vlo + k * (2048 >> 4), dv0.hi, IDESC_O,
+                   k > 0 ? 1u : acc0);
         }
       };
       bool ok = mbar_wait(bar_q, 0, abort_flag, 0x201) &&
@@ -271,21 +291,25 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ---------------------------------------------------------- softmax warps
-    const int t = warp >> 2;              // query tile of this warpgroup
+    const int t = warp >> 3;              // query tile of this warpgroup
+    const int h = (warp >> 2) & 1;        // key half: keys [64h, 64h+64) of each tile
     const int row = threadIdx.x & 127;    // TMEM lane
     const int qt = t ? qt1 : qt0;
     const int n_t = t ? n1 : n0;
     const int qrow = qt * C::BM + row;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t scol = t ? C::COL_S1 : C::COL_S0;
-    const uint32_t ocol = t ? C::COL_O1 : C::COL_O0;
+    const uint32_t scol = (t ? C::COL_S1 : C::COL_S0) + 64 * h;  // this half's scores
+    constexpr int DH = D / 2;                                    // O columns per half
+    const uint32_t ocol = (t ? C::COL_O1 : C::COL_O0) + DH * h;
+    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX) + t * 512 + row;  // + slot*256 + half*128
+    float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM) + t * 512 + row;  // + half*256 + which*128
     const float c = p.scale_log2;
-    float m = -INFINITY;  // reference max of c * s, base-2 units
-    float l = 0.f;        // row sum of the weights 2^(c s - m)
+    float m = -INFINITY;  // reference max of c * s, base-2 units (same in both halves)
+    float l = 0.f;        // this half's row sum of the weights 2^(c s - m)
     float lr = 0.f;       // the same sum over the weights rounded to bf16
     bool ok = true;
 #ifdef FA2_TRACE
-    const bool trace_row = trace_cta && row == 0;
+    const bool trace_row = trace_cta && row == 0 && h == 0;
 #endif
     for (int j = 0; j < n_t; ++j) {
       FA2_TRACE_AT(trace_row, 8 * t + 0, j);
@@ -293,50 +317,54 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) break;
       FA2_TRACE_AT(trace_row, 8 * t + 1, j);
       tc_fence_after();
-      // pass 1: row max over the 128 scores, read from TMEM in two halves
-      const int k0 = j * C::BN;
-      const bool need_mask = (p.causal && j == qt) || (k0 + C::BN > p.N);
+      const int k0 = j * C::BN + 64 * h;  // first key of this half
+      const bool need_mask = (p.causal && j == qt) || (j * C::BN + C::BN > p.N);
       const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys [0, lim) allowed
-      float mx = -INFINITY;
+      float s[64];
+      tmem_ld64(lane_base + scol, s);
+      if (need_mask) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float s[64];
-        tmem_ld64(lane_base + scol + 64 * h, s);
-        if (need_mask) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (k0 + 64 * h + i >= lim) s[i] = -INFINITY;
-        }
+        for (int i = 0; i < 64; ++i)
+          if (k0 + i >= lim) s[i] = -INFINITY;
+      }
+      float mx;
+      {
         float a = s[0], b = s[1];
 #pragma unroll
-        for (int i = 2; i < 64; i += 4) {
+        for (int i = 2; i < 62; i += 4) {
           a = max3(a, s[i], s[i + 1]);
           b = max3(b, s[i + 2], s[i + 3]);
         }
-        mx = max3(mx, a, b);
+        mx = max3(a, b, fmaxf(s[62], s[63]));
       }
+      // row max over both halves: publish this half's, read the other's
+      const int slot = j & 1;
+      xmax[slot * 256 + h * 128] = mx;
+      mbar_arrive(bar_xmax(t, slot));
+      ok = mbar_wait(bar_xmax(t, slot), (j >> 1) & 1, abort_flag, 0x304);
+      if (!ok) break;
+      mx = fmaxf(mx, xmax[slot * 256 + (1 - h) * 128]);
       FA2_TRACE_AT(trace_row, 8 * t + 2, j);
       const float m_cand = fmaxf(m, mx * c);
       const bool grow = m_cand - m > C::RESCALE_THRESHOLD;  // always true for the first tile
       const float alpha = grow ? ex2(m - m_cand) : 1.f;
       if (grow) m = m_cand;
-      // pass 2: weights 2^(c s - m) in pairs, written back over S as bf16 P.
+      // weights 2^(c s - m) in pairs, written back over this half's S as bf16 P.
       // rs: sum of the fp32 weights (for LSE); rr: sum of the bf16-rounded weights
       // that the P V product actually uses (for O / l, so O stays a convex
       // combination of V rows even when one weight dominates)
       const unsigned long long c2 = f2(c, c), negm2 = f2(-m, -m);
       unsigned long long rs2 = f2(0.f, 0.f), rr2 = f2(0.f, 0.f);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float s[64];
-        tmem_ld64(lane_base + scol + 64 * h, s);
-        uint32_t pk[32];
+      for (int q = 0; q < 2; ++q) {
+        uint32_t pk[16];
         if (!need_mask) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < 16; ++i) {
+            const int e = 32 * q + 2 * i;
             float x0, x1, p0, p1;
-            f2_split(f2_fma(f2(s[2 * i], s[2 * i + 1]), c2, negm2), x0, x1);
-            if (i % C::POLY_EVERY == C::POLY_EVERY - 1) {
+            f2_split(f2_fma(f2(s[e], s[e + 1]), c2, negm2), x0, x1);
+            if ((16 * q + i) % C::POLY_EVERY == C::POLY_EVERY - 1) {
               exp2_poly2(x0, x1, p0, p1);  // FMA pipe: balances the MUFU unit
             } else {
               p0 = ex2(x0);
@@ -350,18 +378,19 @@ __global__ void __launch_bounds__(320, 1)
         } else {
           // masked keys contribute exactly 0 (also when c == 0, where -inf * c is NaN)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int kk = k0 + 64 * h + 2 * i;
-            const float p0 = kk >= lim ? 0.f : ex2(fmaf(s[2 * i], c, -m));
-            const float p1 = kk + 1 >= lim ? 0.f : ex2(fmaf(s[2 * i + 1], c, -m));
+          for (int i = 0; i < 16; ++i) {
+            const int e = 32 * q + 2 * i;
+            const float p0 = k0 + e >= lim ? 0.f : ex2(fmaf(s[e], c, -m));
+            const float p1 = k0 + e + 1 >= lim ? 0.f : ex2(fmaf(s[e + 1], c, -m));
             const uint32_t w = pack_bf16(p0, p1);
             pk[i] = w;
             rs2 = f2_add(rs2, f2(p0, p1));
             rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
           }
         }
-        // P for keys [64h, 64h+64) goes to columns [32h, 32h+32): S there is already consumed
-        tmem_st32(lane_base + scol + 32 * h, pk);
+        // P of keys [32q, 32q+32) of this half -> columns [16q, 16q+16): the scores
+        // there are already in registers
+        tmem_st16(lane_base + scol + 16 * q, pk);
       }
       FA2_TRACE_AT(trace_row, 8 * t + 3, j);
       float rs_lo, rs_hi, rr_lo, rr_hi;
@@ -369,10 +398,11 @@ __global__ void __launch_bounds__(320, 1)
       f2_split(rr2, rr_lo, rr_hi);
       l = l * alpha + (rs_lo + rs_hi);
       lr = lr * alpha + (rr_lo + rr_hi);
-      // O holds PV_0..PV_{j-1}: all complete, since S_j was issued after them
+      // O holds PV_0..PV_{j-1}: all complete, since S_j was issued after them.
+      // Each half rescales its own D/2 columns of O.
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-        for (int q = 0; q < D / 32; ++q) {
+        for (int q = 0; q < DH / 32; ++q) {
           float o[32];
           tmem_ld32(lane_base + ocol + 32 * q, o);
           uint32_t u[32];
@@ -388,12 +418,21 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (ok && n_t > 0) ok = mbar_wait(bar_o_done(t), 0, abort_flag, 0x303);
     if (ok) {
+      // row sums over both halves
+      xsum[h * 256] = l;
+      xsum[h * 256 + 128] = lr;
+      mbar_arrive(bar_xsum(t));
+      ok = mbar_wait(bar_xsum(t), 0, abort_flag, 0x305);
+    }
+    if (ok) {
+      l += xsum[(1 - h) * 256];
+      lr += xsum[(1 - h) * 256 + 128];
       tc_fence_after();
       const float inv_l = 1.f / lr;
       const bool store = qrow < p.N;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + qrow) * D;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + qrow) * D + DH * h;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = 0; q < DH / 32; ++q) {
         float o[32];
         tmem_ld32(lane_base + ocol + 32 * q, o);
         uint4 w[4];
@@ -406,7 +445,8 @@ __global__ void __launch_bounds__(320, 1)
           for (int i = 0; i < 4; ++i) dst[i] = w[i];
         }
       }
-      if (store) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * 0.69314718055994530942f;
+      if (store && h == 0)
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * 0.69314718055994530942f;
     }
   }
 
@@ -414,7 +454,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == C::WARP_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fa2
