@@ -145,7 +145,11 @@ struct BwdCfg {
   static_assert(D == 64 || D == 128, "head dim");
   static constexpr int BM = 128;                      // query rows per step
   static constexpr int BN = 128;                      // keys per item
-  static constexpr int STAGES = 2;
+  static constexpr int STAGES = 2;                    // Q (with LSE2 and D) stages
+  // dO stages: dO_i is last read by dV_i in the middle of step i, half a step
+  // before dP of step i+1 needs the next tile, so d = 128 single-buffers it and
+  // spends the 32 KB on the dQ staging buffer
+  static constexpr int DO_STAGES = (D == 128) ? 1 : 2;
   static constexpr int CHUNKS = D / 64;
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int CHUNK_BYTES = 128 * 128;
@@ -154,13 +158,17 @@ struct BwdCfg {
   static constexpr int OFF_V = TILE_BYTES;
   static constexpr int OFF_Q = 2 * TILE_BYTES;                    // + s * TILE_BYTES
   static constexpr int OFF_DO = OFF_Q + STAGES * TILE_BYTES;      // + s * TILE_BYTES
-  static constexpr int OFF_DS = OFF_DO + STAGES * TILE_BYTES;     // 128 x 128 bf16
-  static constexpr int OFF_VEC = OFF_DS + 32768;                  // [s][LSE2 | D]
+  static constexpr int OFF_DS = OFF_DO + DO_STAGES * TILE_BYTES;  // 128 x 128 bf16
+  // dQ staging for the TMA reductions: two 128-byte-swizzled boxes of
+  // [128 query rows][32 fp32], i.e. d columns [0, 64) of one step's dQ tile
+  static constexpr int OFF_STG = OFF_DS + 32768;
+  static constexpr int STG_BOX_BYTES = 16384;
+  static constexpr int OFF_VEC = OFF_STG + 2 * STG_BOX_BYTES;     // [s][LSE2 | D]
   static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
   // kv_full, kv_empty, st_full[S], st_empty[S], s_full, dp_full, p_ready,
   // ds_ready, dsm_free, dq_full, dq_empty, dkv_done, dkv_free, drain,
-  // item_full[2], item_empty[2]
-  static constexpr int NUM_BARS = 2 + 2 * STAGES + 10 + 4;
+  // item_full[2], item_empty[2], do_full[DS], do_empty[DS], staged, stg_free
+  static constexpr int NUM_BARS = 2 + 2 * STAGES + 10 + 4 + 2 * DO_STAGES + 2;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;         // tmem slot, abort, items[2]
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   // d = 128 uses 231,6xx bytes: there is no room for alignment slack, so the
@@ -169,9 +177,13 @@ struct BwdCfg {
   static constexpr int SMEM_ALLOC = NEEDS_ALIGNED_BASE ? SMEM_BYTES : SMEM_BYTES + 1024;
   static constexpr int NWG = 4;                       // elementwise warpgroups
   static constexpr int CW = 128 / NWG;                 // query columns per group
-  static constexpr int WARP_TMA = 4 * NWG, WARP_MMA = 4 * NWG + 1;
-  static constexpr int THREADS = 32 * (4 * NWG + 2);
+  static constexpr int WARP_TMA = 4 * NWG, WARP_MMA = 4 * NWG + 1, WARP_RED = 4 * NWG + 2;
+  static constexpr int THREADS = 32 * (4 * NWG + 3);
   static constexpr int ELEM_THREADS = 128 * NWG;
+  // threads that stage dQ for the TMA reductions: d = 128, the warps whose
+  // TMEM lanes (d rows of dQ^T) are [0, 64); d = 64, all (each group its own
+  // 16 d columns). The other d = 128 warps reduce their rows with red.global.
+  static constexpr int STG_THREADS = (D == 128) ? ELEM_THREADS / 2 : ELEM_THREADS;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   // dQ layout: d = 128 computes dQ^T (d on lanes), so each warp reduction adds
@@ -238,12 +250,13 @@ __device__ __forceinline__ void decode_item(int item, int n_ktiles, int BH, int 
 }
 
 // WITH_DQ = false is the dK/dV-only variant used when dQ comes from the
-// separate query-parallel kernel (fa2_bwd_dq_kernel).
+// separate query-parallel kernel (fa2_bwd_dq_kernel). tm_dq maps the fp32 dQ
+// accumulator for the TMA reductions.
 template <int D, bool WITH_DQ>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (C::NEEDS_ALIGNED_BASE && (smem_u32(smem_raw) & 1023u) != 0) {
@@ -276,6 +289,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const uint32_t bar_drain = bar_s_full + 72;
   auto bar_item_full = [&](int q) { return bar_s_full + 80 + 8 * q; };
   auto bar_item_empty = [&](int q) { return bar_s_full + 96 + 8 * q; };
+  auto bar_do_full = [&](int s) { return bar_s_full + 112 + 8 * s; };
+  auto bar_do_empty = [&](int s) { return bar_s_full + 112 + 8 * (C::DO_STAGES + s); };
+  const uint32_t bar_staged = bar_s_full + 112 + 16 * C::DO_STAGES;
+  const uint32_t bar_stg_free = bar_staged + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* item_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
@@ -300,8 +317,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_init(bar_drain, 1);
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar_item_full(q), 1);
-      mbar_init(bar_item_empty(q), 1 + C::ELEM_THREADS);  // MMA thread + elementwise threads
+      // MMA thread + elementwise threads + reduction thread
+      mbar_init(bar_item_empty(q), 2 + C::ELEM_THREADS);
     }
+    for (int s = 0; s < C::DO_STAGES; ++s) {
+      mbar_init(bar_do_full(s), 1);
+      mbar_init(bar_do_empty(s), 1);
+    }
+    mbar_init(bar_staged, C::STG_THREADS);
+    mbar_init(bar_stg_free, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -314,6 +338,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_do);
+    prefetch_tensormap(&tm_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -335,6 +360,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     if (lane == 0) {
       int last_st_parity[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) last_st_parity[s] = -1;
+      int last_do_parity[C::DO_STAGES];
+      for (int s = 0; s < C::DO_STAGES; ++s) last_do_parity[s] = -1;
       int last_kv_parity = -1;
       bool ok = true;
       int gs = 0;
@@ -368,24 +395,33 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             last_kv_parity = n & 1;
           }
           const uint32_t bar = bar_st_full(s);
-          mbar_arrive_expect_tx(bar, 2 * C::TILE_BYTES + 2 * C::VEC_BYTES);
-          for (int c = 0; c < C::CHUNKS; ++c) {
+          mbar_arrive_expect_tx(bar, C::TILE_BYTES + 2 * C::VEC_BYTES);
+          for (int c = 0; c < C::CHUNKS; ++c)
             tma_load_3d(sbase + C::OFF_Q + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar,
                         c * 64, i * C::BM, bh);
-            tma_load_3d(sbase + C::OFF_DO + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do, bar,
-                        c * 64, i * C::BM, bh);
-          }
           const size_t voff = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * C::BM;
           const uint32_t vec = sbase + C::OFF_VEC + s * 2 * C::VEC_BYTES;
           bulk_load(vec, p.lse2 + voff, C::VEC_BYTES, bar);
           bulk_load(vec + C::VEC_BYTES, p.delta + voff, C::VEC_BYTES, bar);
           last_st_parity[s] = (gs / C::STAGES) & 1;
+          // dO_i once dV of the step that last used this dO buffer is done
+          const int ds = gs % C::DO_STAGES;
+          if (gs >= C::DO_STAGES)
+            ok = mbar_wait(bar_do_empty(ds), ((gs / C::DO_STAGES) - 1) & 1, abort_flag, 0x1105);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar_do_full(ds), C::TILE_BYTES);
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_3d(sbase + C::OFF_DO + ds * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do,
+                        bar_do_full(ds), c * 64, i * C::BM, bh);
+          last_do_parity[ds] = (gs / C::DO_STAGES) & 1;
         }
       }
       // never leave the CTA with copies still landing in its shared memory
       if (last_kv_parity >= 0) mbar_wait(bar_kv_full, last_kv_parity, abort_flag, 0x1102);
       for (int s = 0; s < C::STAGES; ++s)
         if (last_st_parity[s] >= 0) mbar_wait(bar_st_full(s), last_st_parity[s], abort_flag, 0x1103);
+      for (int s = 0; s < C::DO_STAGES; ++s)
+        if (last_do_parity[s] >= 0) mbar_wait(bar_do_full(s), last_do_parity[s], abort_flag, 0x1106);
     }
   } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
@@ -440,7 +476,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             tc_fence_after();
           }
           FA2_TRACE_AT(trace_cta && n == 0, 17, it);
-          const uint32_t dolo = dOk.lo + s * TILE16;
+          const int ds = g % C::DO_STAGES;
+          ok = mbar_wait(bar_do_full(ds), (g / C::DO_STAGES) & 1, abort_flag, 0x120B);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t dolo = dOk.lo + ds * TILE16;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)  // dP^T = V dO_i^T
             umma_ss2(tmem + C::COL_DP, dV.lo + kmaj(k), dV.hi, dolo + kmaj(k), dOk.hi, IDESC_SS,
@@ -455,7 +495,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           }
           FA2_TRACE_AT(trace_cta && n == 0, 18, it);
           tc_fence_after();
-          const uint32_t domlo = dOm.lo + s * TILE16;
+          const uint32_t domlo = dOm.lo + ds * TILE16;
 #pragma unroll
           for (int k = 0; k < C::BM / 16; ++k) {
             // queries 16k..16k+15 sit in group g = 16k / CW at column CW g + (16k mod CW) / 2
@@ -463,6 +503,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             umma_ts2(tmem + C::COL_DV, tmem + pcol, domlo + k * (2048 >> 4), dOm.hi, IDESC_KV,
                      k > 0 ? 1u : acc0);
           }
+          umma_commit(bar_do_empty(ds));  // dV was the last reader of dO_i
           if (it + 1 < n_iter) {
             ok = mbar_wait(bar_st_full((g + 1) % C::STAGES), ((g + 1) / C::STAGES) & 1, abort_flag,
                            0x1208);
@@ -508,6 +549,38 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       umma_commit(bar_drain);
       mbar_wait(bar_drain, 0, abort_flag, 0x1207);
     }
+  } else if (warp == C::WARP_RED) {
+    // ---------------------------------------------------------- dQ reductions
+    // Once the staging threads have written d columns [0, 64) of step g's dQ
+    // tile to the staging buffer, one thread has the TMA add it into the fp32
+    // accumulator and frees the buffer as soon as the TMA has read it.
+    if (lane == 0 && WITH_DQ) {
+      bool ok = true;
+      int gs = 0;
+      for (int n = 0; ok; ++n) {
+        const int item = take_item(n, 0x1709);
+        if (item < 0) break;
+        int ktile, bh;
+        decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
+        const int i_first = p.causal ? ktile : 0;
+        const int n_iter = steps_of(ktile);
+        for (int it = 0; it < n_iter; ++it) {
+          const int g = gs + it;
+          ok = mbar_wait(bar_staged, g & 1, abort_flag, 0x1701);
+          if (!ok) break;
+          tma_reduce_add_3d(&tm_dq, sbase + C::OFF_STG, 0, (i_first + it) * C::BM, bh);
+          tma_reduce_add_3d(&tm_dq, sbase + C::OFF_STG + C::STG_BOX_BYTES, 32, (i_first + it) * C::BM, bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(bar_stg_free);
+        }
+        gs += n_iter;
+      }
+      bulk_wait_group0();  // every reduction has landed before the kernel ends
+    } else if (lane == 0) {
+      for (int n = 0;; ++n)  // dK/dV only: take part in the item hand-off, nothing else
+        if (take_item(n, 0x1709) < 0) break;
+    }
   } else {
     // ------------------------------------------------ elementwise groups (0-15)
     constexpr int CW = C::CW;
@@ -528,36 +601,62 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #ifdef FA2_TRACE
       const bool trace_row = trace_cta && n == 0 && r == 0 && g < 2;
 #endif
-      // dQ of step it (this group's share) -> fp32 accumulator. The TMEM columns
-      // are released as soon as the values are in registers; the reductions follow.
+      // dQ of step it (this group's share) -> fp32 accumulator: d columns [0, 64)
+      // through the staging buffer and the TMA, the rest (d = 128) with
+      // red.global. The TMEM columns are released as soon as the values are in
+      // registers.
+      const uint32_t stg = sbase + C::OFF_STG;
       auto drain = [&](int it) -> bool {
         if (!mbar_wait(bar_dq_full, (gs + it) & 1, abort_flag, 0x1304)) return false;
         FA2_TRACE_AT(trace_row, 8 * g + 4, it);
         tc_fence_after();
         float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i_first + it) * C::BM) * D;
+        const int gg = gs + it;
         if constexpr (C::DQ_T) {
-          // lane r holds dQ^T[d = r][query CW g + q]: each warp instruction adds 32
-          // consecutive d values of one query row (128 contiguous bytes)
+          // lane r holds dQ^T[d = r][query CW g + q]
           float v[CW];
           tmem_ld32(lane_base + C::COL_DQ + CW * g, v);
           tc_fence_before();
           mbar_arrive(bar_dq_empty);
-          float* col = acc + static_cast<size_t>(CW * g) * D + r;
+          if (r < 64) {
+            // staged: row q of box r/32 holds query CW g + q; d = r sits in 16-byte
+            // unit ((r mod 32) / 4) xor (row mod 8) of the 128-byte swizzle
+            if (gg > 0 && !mbar_wait(bar_stg_free, (gg - 1) & 1, abort_flag, 0x1306)) return false;
+            const uint32_t box = stg + (r >> 5) * C::STG_BOX_BYTES;
+            const uint32_t unit = static_cast<uint32_t>((r & 31) >> 2);
+            const uint32_t word = static_cast<uint32_t>(r & 3) * 4;
 #pragma unroll
-          for (int q = 0; q < CW; ++q) red_add(col + static_cast<size_t>(q) * D, v[q]);
+            for (int q = 0; q < CW; ++q) {
+              const int row = CW * g + q;
+              st_shared_f32(box + row * 128 + ((unit ^ (row & 7)) << 4) + word, v[q]);
+            }
+            fence_async_smem();
+            mbar_arrive(bar_staged);
+          } else {
+            // each warp instruction adds 32 consecutive d values of one query row
+            float* col = acc + static_cast<size_t>(CW * g) * D + r;
+#pragma unroll
+            for (int q = 0; q < CW; ++q) red_add(col + static_cast<size_t>(q) * D, v[q]);
+          }
         } else {
-          // lane r holds dQ[query r][d]; this group adds d columns [g D/4, (g+1) D/4)
+          // lane r holds dQ[query r][d]; this group stages d columns [16 g, 16 g + 16)
           constexpr int DW = D / C::NWG;
+          static_assert(DW == 16, "d = 64 stages all of dQ");
           float v[DW];
-          if constexpr (DW == 32)
-            tmem_ld32(lane_base + C::COL_DQ + DW * g, v);
-          else
-            tmem_ld16(lane_base + C::COL_DQ + DW * g, v);
+          tmem_ld16(lane_base + C::COL_DQ + DW * g, v);
           tc_fence_before();
           mbar_arrive(bar_dq_empty);
-          float* row = acc + static_cast<size_t>(r) * D + DW * g;
+          if (gg > 0 && !mbar_wait(bar_stg_free, (gg - 1) & 1, abort_flag, 0x1306)) return false;
 #pragma unroll
-          for (int e = 0; e < DW; e += 4) red_add_v4(row + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
+          for (int u = 0; u < DW / 4; ++u) {
+            const int col = DW * g + 4 * u;
+            const uint32_t box = stg + (col >> 5) * C::STG_BOX_BYTES;
+            const uint32_t unit = static_cast<uint32_t>((col & 31) >> 2);
+            st_shared_v4(box + r * 128 + ((unit ^ (r & 7)) << 4), v[4 * u], v[4 * u + 1], v[4 * u + 2],
+                         v[4 * u + 3]);
+          }
+          fence_async_smem();
+          mbar_arrive(bar_staged);
         }
         FA2_TRACE_AT(trace_row, 8 * g + 5, it);
         return true;

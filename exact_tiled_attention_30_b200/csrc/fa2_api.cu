@@ -59,6 +59,23 @@ bool make_map_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, int
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over the fp32 dQ accumulator [BH, Np, d] seen as 3-D (d, Np, BH),
+// box = 32 elements of d (128 bytes) x 128 rows x 1 head, 128-byte swizzle: the
+// backward kernel adds staged dQ tiles into it with TMA reductions.
+bool make_map_acc(CUtensorMap* map, float* base, int BH, int Np, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Np),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(Np) * d * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Current device must be compute capability 10.0 (B200 class, sm_100a code).
 fa2_status check_device(int* dev_out) {
   int dev = 0;
@@ -208,9 +225,10 @@ fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const vo
     if (st != FA2_OK) return st;
   }
   const WsLayout w = ws_layout(workspace, BH, N, D);
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!make_map_bhnd(&tq, q, BH, N, D, 128) || !make_map_bhnd(&tk, k, BH, N, D, 128) ||
-      !make_map_bhnd(&tv, v, BH, N, D, 128) || !make_map_bhnd(&tdo, dO, BH, N, D, 128))
+      !make_map_bhnd(&tv, v, BH, N, D, 128) || !make_map_bhnd(&tdo, dO, BH, N, D, 128) ||
+      !make_map_acc(&tdq, w.dq_acc, BH, w.Np, D))
     return FA2_ERR_CUDA;
   fa2::BwdParams bp;
   bp.dk = reinterpret_cast<__nv_bfloat16*>(dk);
@@ -229,7 +247,7 @@ fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const vo
   // persistent: one CTA per SM (its shared memory allows no second one)
   const long long items = static_cast<long long>(bp.n_ktiles) * BH;
   const int ctas = static_cast<int>(items < sm_count(dev) ? items : sm_count(dev));
-  fa2::fa2_bwd_kernel<D, WITH_DQ><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, bp);
+  fa2::fa2_bwd_kernel<D, WITH_DQ><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, tdq, bp);
   return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
 
