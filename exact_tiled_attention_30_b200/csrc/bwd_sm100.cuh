@@ -599,7 +599,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int i_first = p.causal ? ktile : 0;
       const int n_iter = steps_of(ktile);
 #ifdef FA2_TRACE
-      const bool trace_row = trace_cta && n == 0 && r == 0 && g < 2;
+      // group 0: a thread of the first warp (dQ staging at d = 128); group 1: a
+      // thread of the third warp (dQ reductions at d = 128)
+      const bool trace_row = trace_cta && n == 0 && ((g == 0 && r == 0) || (g == 1 && r == 64));
 #endif
       // dQ of step it (this group's share) -> fp32 accumulator: d columns [0, 64)
       // through the staging buffer and the TMA, the rest (d = 128) with
