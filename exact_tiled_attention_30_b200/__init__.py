@@ -77,6 +77,11 @@ def load_library():
     lib.fa2_backward_main_dkdv.restype = i
     lib.fa2_backward_dq.argtypes = [vp] * 5 + [i, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t, vp]
     lib.fa2_backward_dq.restype = i
+    lib.fa2_forward_backward_host_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa2_forward_backward_host_workspace_size.restype = ctypes.c_size_t
+    lib.fa2_forward_backward_host.argtypes = [vp] * 9 + [i, i, i, i, i, ctypes.c_float, i, vp,
+                                                        ctypes.c_size_t, vp]
+    lib.fa2_forward_backward_host.restype = i
     lib.fa2_status_string.argtypes = [i]
     lib.fa2_status_string.restype = ctypes.c_char_p
     lib.fa2_get_device_status.argtypes = [vp, ctypes.POINTER(i)]
@@ -291,3 +296,63 @@ def fa2_backward_noalloc(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale:
     _check("fa2_backward_noalloc", fn(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
         B, H, N, d, int(bool(causal)), float(scale), _stream(stream)))
+
+
+def fa2_forward_backward_host_workspace_size(B: int, H: int, N: int, d: int,
+                                             heads_per_chunk: int = 0) -> int:
+    return int(load_library().fa2_forward_backward_host_workspace_size(B, H, N, d, heads_per_chunk))
+
+
+def _require_host(t, name, dtype):
+    if t.is_cuda or not t.is_contiguous() or t.dtype != dtype:
+        raise ValueError(f"{name} must be a contiguous {dtype} host tensor")
+
+
+def fa2_forward_backward_host(q, k, v, dout, o, lse, dq, dk, dv, causal: bool, scale: float,
+                              workspace, heads_per_chunk: int = 0, stream=None) -> None:
+    """C ABI fa2_forward_backward_host: q, k, v, dout and the outputs o, lse, dq,
+    dk, dv are HOST tensors (page-locked for the copies to overlap); workspace is
+    a CUDA uint8 tensor of fa2_forward_backward_host_workspace_size bytes."""
+    import torch
+
+    B, H, N, d = _bhnd(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (o, "o"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _require_host(t, n, torch.bfloat16)
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
+    _require_host(lse, "lse", torch.float32)
+    if tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be [B, H, N]")
+    _require(workspace, "workspace")
+    _check("fa2_forward_backward_host", load_library().fa2_forward_backward_host(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, H, N, d, int(bool(causal)), float(scale), int(heads_per_chunk), _ptr(workspace),
+        _nbytes(workspace), _stream(stream)))
+
+
+def attention_forward_backward_host(q, k, v, dout, causal: bool = False, scale: float | None = None,
+                                    heads_per_chunk: int = 0, workspace=None, out=None,
+                                    stream=None):
+    """Forward and backward of host tensors, copies pipelined with the kernels.
+    Returns host (o, lse, dq, dk, dv), page-locked (or the tensors of `out`);
+    they are complete once `stream` (default: the current stream) has passed
+    the call."""
+    import torch
+
+    B, H, N, d = _bhnd(q)
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        pin = dict(dtype=torch.bfloat16, pin_memory=True)
+        out = (torch.empty((B, H, N, d), **pin), torch.empty((B, H, N), dtype=torch.float32,
+                                                            pin_memory=True),
+               torch.empty((B, H, N, d), **pin), torch.empty((B, H, N, d), **pin),
+               torch.empty((B, H, N, d), **pin))
+    if workspace is None:
+        workspace = torch.empty(fa2_forward_backward_host_workspace_size(B, H, N, d, heads_per_chunk),
+                                dtype=torch.uint8, device="cuda")
+    o, lse, dq, dk, dv = out
+    fa2_forward_backward_host(q, k, v, dout, o, lse, dq, dk, dv, causal, scale, workspace,
+                              heads_per_chunk, stream)
+    return o, lse, dq, dk, dv

@@ -592,6 +592,164 @@ fa2_status fa2_backward_noalloc(const void* q, const void* k, const void* v, con
 
 }  // extern "C"
 
+// ------------------------------------------------------- host-buffer pipeline
+namespace {
+
+constexpr int kHostSlots = 3;  // chunks in flight
+
+int host_chunk_heads(int BH, int heads_per_chunk) {
+  int c = heads_per_chunk > 0 ? heads_per_chunk : (BH + 7) / 8;
+  return c < 1 ? 1 : (c > BH ? BH : c);
+}
+
+inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Device layout of one slot: q, k, v, dO, o, dq, dk, dv (bf16 [c, N, d] each),
+// lse (fp32 [c, N]), then the backward workspace of c heads.
+struct HostSlot {
+  size_t tensor_bytes, lse_bytes, ws_bytes, bytes;
+};
+
+HostSlot host_slot(int c, int N, int d) {
+  HostSlot h;
+  h.tensor_bytes = round256(static_cast<size_t>(c) * N * d * 2);
+  h.lse_bytes = round256(static_cast<size_t>(c) * N * 4);
+  h.ws_bytes = round256(fa2_backward_workspace_size(1, c, N, d));
+  h.bytes = 8 * h.tensor_bytes + h.lse_bytes + h.ws_bytes;
+  return h;
+}
+
+// Three non-blocking streams (copy in, compute, copy out) and the events that
+// chain a slot through them, created once per device and kept for the process.
+struct HostPipe {
+  cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
+  cudaEvent_t entry = nullptr, exit = nullptr;
+  cudaEvent_t in_done[kHostSlots] = {}, comp_done[kHostSlots] = {}, out_done[kHostSlots] = {};
+  bool used[kHostSlots] = {};
+  bool ready = false;
+};
+
+HostPipe g_host_pipe[kMaxDevices];
+std::mutex g_host_mu;  // serialises enqueueing on the shared streams
+
+fa2_status host_pipe_init(HostPipe& hp) {
+  if (hp.ready) return FA2_OK;
+  bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&hp.comp, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp.entry, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp.exit, cudaEventDisableTiming) == cudaSuccess;
+  for (int i = 0; ok && i < kHostSlots; ++i)
+    ok = cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  hp.ready = true;
+  return FA2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa2_forward_backward_host_workspace_size(int B, int H, int N, int d, int heads_per_chunk) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128) || heads_per_chunk < 0) return 0;
+  const int c = host_chunk_heads(B * H, heads_per_chunk);
+  return kHostSlots * host_slot(c, N, d).bytes;
+}
+
+fa2_status fa2_forward_backward_host(const void* q, const void* k, const void* v, const void* dO,
+                                     void* o, float* lse, void* dq, void* dk, void* dv, int B,
+                                     int H, int N, int d, int causal, float scale,
+                                     int heads_per_chunk, void* device_workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !o || !lse || !dq || !dk || !dv || !device_workspace)
+    return FA2_ERR_INVALID_ARG;
+  if (heads_per_chunk < 0) return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_common(B, H, N, d, scale);
+  if (st != FA2_OK) return st;
+  if (workspace_bytes < fa2_forward_backward_host_workspace_size(B, H, N, d, heads_per_chunk))
+    return FA2_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(device_workspace) & 255u) != 0) return FA2_ERR_MISALIGNED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+
+  const int BH = B * H;
+  const int c = host_chunk_heads(BH, heads_per_chunk);
+  const HostSlot hs = host_slot(c, N, d);
+  const size_t head_elems = static_cast<size_t>(N) * d;  // bf16 elements of one head
+
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostPipe& hp = g_host_pipe[dev];
+  st = host_pipe_init(hp);
+  if (st != FA2_OK) return st;
+  cudaStream_t user = reinterpret_cast<cudaStream_t>(stream);
+  bool ok = cudaEventRecord(hp.entry, user) == cudaSuccess &&
+            cudaStreamWaitEvent(hp.in, hp.entry, 0) == cudaSuccess;
+  const char* hq = static_cast<const char*>(q);
+  const char* hk = static_cast<const char*>(k);
+  const char* hv = static_cast<const char*>(v);
+  const char* hdo = static_cast<const char*>(dO);
+  char* ho = static_cast<char*>(o);
+  char* hdq = static_cast<char*>(dq);
+  char* hdk = static_cast<char*>(dk);
+  char* hdv = static_cast<char*>(dv);
+  for (int h0 = 0, chunk = 0; ok && h0 < BH; h0 += c, ++chunk) {
+    const int slot = chunk % kHostSlots;
+    const int nh = BH - h0 < c ? BH - h0 : c;
+    const size_t tb = static_cast<size_t>(nh) * head_elems * 2;  // bytes of one tensor chunk
+    const size_t off = static_cast<size_t>(h0) * head_elems * 2;
+    char* base = static_cast<char*>(device_workspace) + slot * hs.bytes;
+    char* dt[8];  // q, k, v, dO, o, dq, dk, dv
+    for (int i = 0; i < 8; ++i) dt[i] = base + i * hs.tensor_bytes;
+    float* dlse = reinterpret_cast<float*>(base + 8 * hs.tensor_bytes);
+    void* dws = base + 8 * hs.tensor_bytes + hs.lse_bytes;
+    // copy in, once the outputs of the chunk that used this slot are out
+    if (hp.used[slot]) ok = ok && cudaStreamWaitEvent(hp.in, hp.out_done[slot], 0) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dt[0], hq + off, tb, cudaMemcpyHostToDevice, hp.in) == cudaSuccess &&
+         cudaMemcpyAsync(dt[1], hk + off, tb, cudaMemcpyHostToDevice, hp.in) == cudaSuccess &&
+         cudaMemcpyAsync(dt[2], hv + off, tb, cudaMemcpyHostToDevice, hp.in) == cudaSuccess &&
+         cudaMemcpyAsync(dt[3], hdo + off, tb, cudaMemcpyHostToDevice, hp.in) == cudaSuccess &&
+         cudaEventRecord(hp.in_done[slot], hp.in) == cudaSuccess;
+    // forward + backward of the chunk's heads (as B = 1, H = nh)
+    ok = ok && cudaStreamWaitEvent(hp.comp, hp.in_done[slot], 0) == cudaSuccess;
+    if (!ok) break;
+    st = fa2_forward(dt[0], dt[1], dt[2], dt[4], dlse, 1, nh, N, d, causal, scale, hp.comp);
+    if (st == FA2_OK)
+      st = fa2_backward(dt[0], dt[1], dt[2], dt[4], dlse, dt[3], dt[5], dt[6], dt[7], 1, nh, N, d,
+                        causal, scale, dws, hs.ws_bytes, hp.comp);
+    if (st != FA2_OK) break;
+    ok = cudaEventRecord(hp.comp_done[slot], hp.comp) == cudaSuccess &&
+         cudaStreamWaitEvent(hp.out, hp.comp_done[slot], 0) == cudaSuccess;
+    // copy out
+    const size_t loff = static_cast<size_t>(h0) * N * 4;
+    ok = ok && cudaMemcpyAsync(ho + off, dt[4], tb, cudaMemcpyDeviceToHost, hp.out) == cudaSuccess &&
+         cudaMemcpyAsync(reinterpret_cast<char*>(lse) + loff, dlse, static_cast<size_t>(nh) * N * 4,
+                         cudaMemcpyDeviceToHost, hp.out) == cudaSuccess &&
+         cudaMemcpyAsync(hdq + off, dt[5], tb, cudaMemcpyDeviceToHost, hp.out) == cudaSuccess &&
+         cudaMemcpyAsync(hdk + off, dt[6], tb, cudaMemcpyDeviceToHost, hp.out) == cudaSuccess &&
+         cudaMemcpyAsync(hdv + off, dt[7], tb, cudaMemcpyDeviceToHost, hp.out) == cudaSuccess &&
+         cudaEventRecord(hp.out_done[slot], hp.out) == cudaSuccess;
+    hp.used[slot] = true;
+  }
+  // the caller's stream continues once the last copy out has completed (the
+  // copy-out stream runs the chunks in order)
+  const bool joined = cudaEventRecord(hp.exit, hp.out) == cudaSuccess &&
+                      cudaStreamWaitEvent(user, hp.exit, 0) == cudaSuccess;
+  if (st != FA2_OK) return st;
+  if (!ok || !joined) {
+    cudaGetLastError();
+    return FA2_ERR_CUDA;
+  }
+  return FA2_OK;
+}
+
+}  // extern "C"
+
 #ifdef FA2_TRACE
 // Debug builds only: copies the trace stamps of the last traced launch.
 extern "C" FA2_API int fa2_debug_trace_read(unsigned long long* host, int n) {

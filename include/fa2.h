@@ -187,6 +187,47 @@ FA2_API fa2_status fa2_backward_noalloc(const void* q, const void* k, const void
                                         void* dq, void* dk, void* dv, int B, int H, int N, int d,
                                         int causal, float scale, void* stream);
 
+/*
+ * Forward and backward from HOST buffers: the form of the computation for
+ * callers whose tensors live in host memory (and how end-to-end throughput,
+ * host<->device copies included, is measured). The pages' method itself is the
+ * two device passes above; this only schedules them with the copies.
+ *
+ *  Inputs  q, k, v, dO: host, bf16 [B, H, N, d] contiguous.
+ *  Outputs o (bf16), lse (fp32 [B, H, N]), dq, dk, dv (bf16): host.
+ *  Same mask, scale, d and size rules as fa2_forward / fa2_backward.
+ *
+ * The B*H heads are processed in chunks of `heads_per_chunk` heads (0 = B*H/8
+ * rounded up). Chunk c's inputs are copied in, its forward and backward run,
+ * and its outputs are copied out on three library-owned streams, up to three
+ * chunks in flight, so that the copies in both directions overlap each other
+ * and the kernels. Host buffers should be page-locked (cudaHostAlloc /
+ * cudaHostRegister); with pageable memory the copies are correct but do not
+ * overlap.
+ *
+ * `device_workspace` (caller-owned device memory, 256-byte aligned, at least
+ * fa2_forward_backward_host_workspace_size(B, H, N, d, heads_per_chunk)
+ * bytes) holds the chunks' device copies and backward workspaces.
+ *
+ * Ordering: the work starts after everything enqueued on `stream` before the
+ * call and the call returns as soon as it is enqueued; work enqueued on
+ * `stream` afterwards (a synchronisation, a read of the outputs) runs after all
+ * of it has completed, copies to host included. Calls on one device are
+ * serialised internally (they share the library's streams); do not let the
+ * host arrays or the workspace change until `stream` has passed the call.
+ * Errors: FA2_ERR_INVALID_ARG (null pointer, heads_per_chunk < 0, workspace too
+ * small), FA2_ERR_MISALIGNED (workspace), FA2_ERR_UNSUPPORTED (d, sizes,
+ * device), FA2_ERR_CUDA (a copy or launch failed; outputs then undefined).
+ */
+FA2_API size_t fa2_forward_backward_host_workspace_size(int B, int H, int N, int d,
+                                                        int heads_per_chunk);
+FA2_API fa2_status fa2_forward_backward_host(const void* q, const void* k, const void* v,
+                                             const void* dO, void* o, float* lse, void* dq,
+                                             void* dk, void* dv, int B, int H, int N, int d,
+                                             int causal, float scale, int heads_per_chunk,
+                                             void* device_workspace, size_t workspace_bytes,
+                                             void* stream);
+
 /* Static, NUL-terminated name of a status code. */
 FA2_API const char* fa2_status_string(int status);
 

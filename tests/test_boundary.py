@@ -135,3 +135,46 @@ def test_backward_ex_rejects_bad_strategy(lib):
     assert lib.fa2_backward_dq_strategy(1, 1, 128, 64, 0) in (1, 2)
     assert lib.fa2_backward_dq(None, A, A, A, A, 1, 1, 128, 64, 0, ctypes.c_float(0.1), A, ws, None) == 1
     assert lib.fa2_backward_main_dkdv(A, A, A, A, A, A, 1, 1, 128, 64, 0, ctypes.c_float(0.1), A, 8, None) == 1
+
+
+def test_host_path_workspace_size(lib):
+    """Three chunk slots of: 8 bf16 tensors + fp32 LSE + the chunk's backward workspace,
+    each rounded up to 256 bytes; heads_per_chunk 0 means ceil(B*H / 8)."""
+    def r256(x):
+        return (x + 255) // 256 * 256
+
+    def expect(B, H, N, d, hpc):
+        c = hpc if hpc > 0 else (B * H + 7) // 8
+        c = max(1, min(c, B * H))
+        slot = (8 * r256(c * N * d * 2) + r256(c * N * 4)
+                + r256(lib.fa2_backward_workspace_size(1, c, N, d)))
+        return 3 * slot
+
+    for args in [(2, 3, 129, 64, 2), (2, 3, 129, 64, 0), (8, 16, 2048, 128, 0), (1, 5, 1, 128, 9),
+                 (1, 1, 300, 64, 1)]:
+        assert lib.fa2_forward_backward_host_workspace_size(*args) == expect(*args), args
+    assert lib.fa2_forward_backward_host_workspace_size(1, 1, 128, 64, -1) == 0
+    assert lib.fa2_forward_backward_host_workspace_size(1, 1, 128, 32, 0) == 0
+
+
+def host(lib, ptrs=None, B=1, H=2, N=128, d=64, scale=0.125, hpc=0, ws_bytes=None):
+    p = [A] * 10 if ptrs is None else ptrs
+    if ws_bytes is None:
+        ws_bytes = lib.fa2_forward_backward_host_workspace_size(B, H, N, d, max(hpc, 0))
+    return lib.fa2_forward_backward_host(*p[:9], B, H, N, d, 1, ctypes.c_float(scale), hpc, p[9],
+                                         ws_bytes, None)
+
+
+def test_host_path_rejects_bad_arguments(lib):
+    for i in range(10):
+        p = [A] * 10
+        p[i] = None
+        assert host(lib, p) == 1, i
+    assert host(lib, hpc=-1) == 1
+    assert host(lib, ws_bytes=1000) == 1
+    assert host(lib, N=0) == 1
+    assert host(lib, scale=float("nan")) == 1
+    assert host(lib, d=80) == 2
+    p = [A] * 10
+    p[9] = A + 16  # the device workspace must be 256-byte aligned
+    assert host(lib, p) == 3
