@@ -773,20 +773,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
         tc_fence_before();
         mbar_arrive(bar_dkv_free);
-        if (store) {
-          uint4 o[DW / 8];
-          uint32_t* ou = reinterpret_cast<uint32_t*>(o);
+        // rows on lanes: transposed in groups of lanes so that every store
+        // instruction writes whole 2*DW-byte row segments
+        const unsigned int rows = __ballot_sync(0xffffffffu, store);
+        const size_t off0 = off - static_cast<size_t>(r & 31) * D;  // lane 0's row
+        uint4 o[DW / 8];
+        uint32_t* ou = reinterpret_cast<uint32_t*>(o);
 #pragma unroll
-          for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-          uint4* dst = reinterpret_cast<uint4*>(p.dv + off);
+        for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+        store_rows_coalesced<DW / 8>(reinterpret_cast<char*>(p.dv + off0), static_cast<size_t>(D) * 2, o, rows);
 #pragma unroll
-          for (int e = 0; e < DW / 8; ++e) dst[e] = o[e];
-#pragma unroll
-          for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(w[2 * e] * p.scale, w[2 * e + 1] * p.scale);
-          dst = reinterpret_cast<uint4*>(p.dk + off);
-#pragma unroll
-          for (int e = 0; e < DW / 8; ++e) dst[e] = o[e];
-        }
+        for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(w[2 * e] * p.scale, w[2 * e + 1] * p.scale);
+        store_rows_coalesced<DW / 8>(reinterpret_cast<char*>(p.dk + off0), static_cast<size_t>(D) * 2, o, rows);
       }
       gs += n_iter;
     }

@@ -126,6 +126,42 @@ fa2_status ensure_smem(KernelT kernel, int bytes, int dev, bool* done) {
   return FA2_OK;
 }
 
+int sm_count(int dev);
+
+// Work-item counters of the persistent forward kernel: a ring of them per
+// device, one per launch, zeroed on the launch's stream right before it. Launches
+// that overlap on the GPU (different streams) use different counters as long as
+// fewer than kFwdCounters of them are in flight at once.
+constexpr unsigned int kFwdCounters = 256;
+__device__ unsigned int g_fwd_counters[kFwdCounters];
+
+unsigned int* fwd_counter(int dev, cudaStream_t stream, fa2_status* st) {
+  static unsigned int* base[kMaxDevices] = {nullptr};
+  static unsigned int next[kMaxDevices] = {0};
+  static std::mutex mu;
+  unsigned int* c = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!base[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_fwd_counters) != cudaSuccess || ptr == nullptr) {
+        cudaGetLastError();
+        *st = FA2_ERR_CUDA;
+        return nullptr;
+      }
+      base[dev] = static_cast<unsigned int*>(ptr);
+    }
+    c = base[dev] + (next[dev]++ % kFwdCounters);
+  }
+  if (cudaMemsetAsync(c, 0, sizeof(unsigned int), stream) != cudaSuccess) {
+    cudaGetLastError();
+    *st = FA2_ERR_CUDA;
+    return nullptr;
+  }
+  *st = FA2_OK;
+  return c;
+}
+
 template <int D>
 fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                           int H, int N, int causal, float scale, cudaStream_t stream, int dev) {
@@ -151,8 +187,13 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.BH = BH;
-  const dim3 grid = p.causal ? dim3(BH * p.n_pairs) : dim3(p.n_pairs, BH);
-  fa2::fa2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  fa2_status st = FA2_OK;
+  p.counter = fwd_counter(dev, stream, &st);
+  if (st != FA2_OK) return st;
+  // persistent: one CTA per SM (its shared memory and TMEM allow no second one)
+  const long long items = static_cast<long long>(BH) * p.n_pairs;
+  const int ctas = static_cast<int>(items < sm_count(dev) ? items : sm_count(dev));
+  fa2::fa2_fwd_kernel<D><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
   return FA2_OK;
 }

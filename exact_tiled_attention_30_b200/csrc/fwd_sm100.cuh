@@ -59,10 +59,11 @@ struct FwdCfg {
   static constexpr int OFF_K = 2 * TILE_BYTES;        // + s * 2 * TILE_BYTES
   static constexpr int OFF_V = 3 * TILE_BYTES;        // + s * 2 * TILE_BYTES
   static constexpr int OFF_BAR = TILE_BYTES * (2 + 2 * STAGES);
-  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain,
-  // xmax[2 tiles][2 slots], xsum[2 tiles]
-  static constexpr int NUM_BARS = 1 + 2 * STAGES + 7 + 6;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;  // tmem slot, abort flag
+  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2],
+  // o_free[2], drain, xmax[2 tiles][2 slots], xsum[2 tiles], item_full[2],
+  // item_empty[2]
+  static constexpr int NUM_BARS = 2 + 2 * STAGES + 9 + 6 + 4;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;  // tmem slot, abort flag, items[2]
   // exchange between the two halves of a row: partial maxima [tile][slot][half][row]
   // and, at the end, partial sums [tile][half][l | lr][row]
   static constexpr int OFF_XMAX = OFF_MISC + 16;
@@ -83,6 +84,7 @@ struct FwdCfg {
 struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
+  unsigned int* counter;  // next work item, zero at launch
   int N;
   int n_qtiles;  // ceil(N / 128)
   int n_pairs;   // ceil(n_qtiles / 2)
@@ -91,6 +93,29 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e)
 };
 
+// Work item -> (pair of query tiles, batch*head). Non-causal: the pairs of one
+// head are consecutive, so they run together and share its K/V tiles in L2.
+// Causal: groups of HEAD_GROUP heads (their K/V stay in L2 while the group
+// runs); inside a group the heaviest pairs of every head come first.
+__device__ __forceinline__ void fwd_decode_item(int item, int n_pairs, int BH, int head_group,
+                                                bool causal, int& pair, int& bh) {
+  if (!causal) {
+    bh = item / n_pairs;
+    pair = item - bh * n_pairs;
+    return;
+  }
+  const int group_items = head_group * n_pairs;
+  const int grp = item / group_items;
+  const int r = item - grp * group_items;
+  const int heads = min(head_group, BH - grp * head_group);
+  pair = n_pairs - 1 - r / heads;
+  bh = grp * head_group + r % heads;
+}
+
+// Persistent: one CTA per SM takes work items (pairs of query tiles) from a
+// counter until none are left. Every barrier phase is counted over the CTA's
+// whole sequence of items: `n` counts items, `kg` key tiles loaded, `jt[t]`
+// key tiles of query tile t.
 template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -102,47 +127,38 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Blocks launch in linear order. Non-causal: grid (pair, batch*head), so the
-  // pairs of one head run together and share its K/V tiles in L2. Causal: a 1-D
-  // grid in groups of HEAD_GROUP heads (their K/V stay in L2 while the group
-  // runs); inside a group the heaviest pairs of every head start first.
-  int pair, bh;
-  if (!p.causal) {
-    pair = blockIdx.x;
-    bh = blockIdx.y;
-  } else {
-    const int group_blocks = C::HEAD_GROUP * p.n_pairs;
-    const int grp = static_cast<int>(blockIdx.x) / group_blocks;
-    const int r = static_cast<int>(blockIdx.x) - grp * group_blocks;
-    const int heads = min(C::HEAD_GROUP, p.BH - grp * C::HEAD_GROUP);
-    pair = p.n_pairs - 1 - r / heads;
-    bh = grp * C::HEAD_GROUP + r % heads;
-  }
+  const int n_items = p.n_pairs * p.BH;
   const int n_kv_total = (p.N + C::BN - 1) / C::BN;
   // query tiles 2*pair and 2*pair+1; with causal masking tile t sees key tiles [0, qt_t]
-  const int qt0 = 2 * pair;
-  const int qt1 = 2 * pair + 1;
-  const int n0 = p.causal ? min(n_kv_total, qt0 + 1) : n_kv_total;
-  const int n1 = p.causal ? min(n_kv_total, qt1 + 1) : n_kv_total;  // n1 >= n0
+  auto tiles_of = [&](int pair, int& n0, int& n1) {
+    n0 = p.causal ? min(n_kv_total, 2 * pair + 1) : n_kv_total;
+    n1 = p.causal ? min(n_kv_total, 2 * pair + 2) : n_kv_total;  // n1 >= n0
+  };
 #ifdef FA2_TRACE
-  const bool trace_cta = p.causal ? blockIdx.x == 7 : (blockIdx.x == 0 && blockIdx.y == 7);
+  const bool trace_cta = blockIdx.x == 7;
 #endif
 
-  const uint32_t bar_q = sbase + C::OFF_BAR;
-  auto bar_kv_full = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + s); };
-  auto bar_kv_empty = [&](int s) { return sbase + C::OFF_BAR + 8 * (1 + C::STAGES + s); };
-  const uint32_t bar_base = sbase + C::OFF_BAR + 8 * (1 + 2 * C::STAGES);
+  const uint32_t bar_q_full = sbase + C::OFF_BAR;
+  const uint32_t bar_q_empty = bar_q_full + 8;
+  auto bar_kv_full = [&](int s) { return sbase + C::OFF_BAR + 8 * (2 + s); };
+  auto bar_kv_empty = [&](int s) { return sbase + C::OFF_BAR + 8 * (2 + C::STAGES + s); };
+  const uint32_t bar_base = sbase + C::OFF_BAR + 8 * (2 + 2 * C::STAGES);
   auto bar_s_full = [&](int t) { return bar_base + 8 * t; };
   auto bar_p_full = [&](int t) { return bar_base + 16 + 8 * t; };
   auto bar_o_done = [&](int t) { return bar_base + 32 + 8 * t; };
-  const uint32_t bar_drain = bar_base + 48;
-  auto bar_xmax = [&](int t, int slot) { return bar_base + 56 + 16 * t + 8 * slot; };
-  auto bar_xsum = [&](int t) { return bar_base + 88 + 8 * t; };
+  auto bar_o_free = [&](int t) { return bar_base + 48 + 8 * t; };
+  const uint32_t bar_drain = bar_base + 64;
+  auto bar_xmax = [&](int t, int slot) { return bar_base + 72 + 16 * t + 8 * slot; };
+  auto bar_xsum = [&](int t) { return bar_base + 104 + 8 * t; };
+  auto bar_item_full = [&](int q) { return bar_base + 120 + 8 * q; };
+  auto bar_item_empty = [&](int q) { return bar_base + 136 + 8 * q; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_empty, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(bar_kv_full(s), 1);
       mbar_init(bar_kv_empty(s), 1);
@@ -151,11 +167,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       mbar_init(bar_s_full(t), 1);
       mbar_init(bar_p_full(t), 256);
       mbar_init(bar_o_done(t), 1);
+      mbar_init(bar_o_free(t), 256);
       mbar_init(bar_xmax(t, 0), 256);
       mbar_init(bar_xmax(t, 1), 256);
       mbar_init(bar_xsum(t), 256);
     }
     mbar_init(bar_drain, 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(bar_item_full(q), 1);
+      mbar_init(bar_item_empty(q), 1 + 512);  // MMA thread + softmax threads
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -173,34 +194,61 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Consumers read item n from the two-slot ring (-1 ends the sequence).
+  auto take_item = [&](int n, int site) -> int {
+    if (!mbar_wait(bar_item_full(n & 1), (n >> 1) & 1, abort_flag, site)) return -1;
+    const int item = item_slot[n & 1];
+    mbar_arrive(bar_item_empty(n & 1));
+    return item;
+  };
+
   if (warp == C::WARP_TMA) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------- scheduler + TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
-      for (int c = 0; c < C::CHUNKS; ++c) {
-        tma_load_3d(sbase + C::OFF_Q + c * C::CHUNK_BYTES, &tm_q, bar_q, c * 64, qt0 * C::BM, bh);
-        tma_load_3d(sbase + C::OFF_Q + C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar_q, c * 64,
-                    qt1 * C::BM, bh);
-      }
       int last_parity[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) last_parity[s] = -1;
+      int last_q_parity = -1;
       bool ok = true;
-      for (int j = 0; j < n1 && ok; ++j) {
-        const int s = j % C::STAGES;
-        const int n = j / C::STAGES;
-        if (n > 0) ok = mbar_wait(bar_kv_empty(s), (n - 1) & 1, abort_flag, 0x101);
+      int kg = 0;  // key tiles loaded so far
+      for (int n = 0; ok; ++n) {
+        int item = static_cast<int>(atomicAdd(p.counter, 1u));
+        if (item >= n_items) item = -1;
+        if (n >= 2) ok = mbar_wait(bar_item_empty(n & 1), ((n >> 1) - 1) & 1, abort_flag, 0x104);
         if (!ok) break;
-        const uint32_t kdst = sbase + C::OFF_K + s * 2 * C::TILE_BYTES;
-        const uint32_t vdst = sbase + C::OFF_V + s * 2 * C::TILE_BYTES;
-        mbar_arrive_expect_tx(bar_kv_full(s), 2 * C::TILE_BYTES);
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(kdst + c * C::CHUNK_BYTES, &tm_k, bar_kv_full(s), c * 64, j * C::BN, bh);
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(vdst + c * C::CHUNK_BYTES, &tm_v, bar_kv_full(s), c * 64, j * C::BN, bh);
-        last_parity[s] = n & 1;
+        item_slot[n & 1] = item;
+        mbar_arrive(bar_item_full(n & 1));
+        if (item < 0) break;
+        int pair, bh, n0, n1;
+        fwd_decode_item(item, p.n_pairs, p.BH, C::HEAD_GROUP, p.causal != 0, pair, bh);
+        tiles_of(pair, n0, n1);
+        // Q0, Q1 once the previous item's S MMAs are done with the buffers
+        if (n >= 1) ok = mbar_wait(bar_q_empty, (n - 1) & 1, abort_flag, 0x105);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_q_full, 2 * C::TILE_BYTES);
+        for (int c = 0; c < C::CHUNKS; ++c) {
+          tma_load_3d(sbase + C::OFF_Q + c * C::CHUNK_BYTES, &tm_q, bar_q_full, c * 64,
+                      2 * pair * C::BM, bh);
+          tma_load_3d(sbase + C::OFF_Q + C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar_q_full,
+                      c * 64, (2 * pair + 1) * C::BM, bh);
+        }
+        last_q_parity = n & 1;
+        for (int j = 0; j < n1 && ok; ++j, ++kg) {
+          const int s = kg % C::STAGES;
+          const int u = kg / C::STAGES;
+          if (u > 0) ok = mbar_wait(bar_kv_empty(s), (u - 1) & 1, abort_flag, 0x101);
+          if (!ok) break;
+          const uint32_t kdst = sbase + C::OFF_K + s * 2 * C::TILE_BYTES;
+          const uint32_t vdst = sbase + C::OFF_V + s * 2 * C::TILE_BYTES;
+          mbar_arrive_expect_tx(bar_kv_full(s), 2 * C::TILE_BYTES);
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_3d(kdst + c * C::CHUNK_BYTES, &tm_k, bar_kv_full(s), c * 64, j * C::BN, bh);
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_3d(vdst + c * C::CHUNK_BYTES, &tm_v, bar_kv_full(s), c * 64, j * C::BN, bh);
+          last_parity[s] = u & 1;
+        }
       }
       // never leave the CTA with copies still landing in its shared memory
-      mbar_wait(bar_q, 0, abort_flag, 0x102);
+      if (last_q_parity >= 0) mbar_wait(bar_q_full, last_q_parity, abort_flag, 0x102);
       for (int s = 0; s < C::STAGES; ++s)
         if (last_parity[s] >= 0) mbar_wait(bar_kv_full(s), last_parity[s], abort_flag, 0x103);
     }
@@ -215,8 +263,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const SDesc dk0 = sdesc_make(sbase + C::OFF_K, 16, 1024);
       const SDesc dv0 = sdesc_make(sbase + C::OFF_V, C::CHUNK_BYTES, 1024);
       constexpr uint32_t STAGE16 = 2 * C::TILE_BYTES / 16;  // stage stride in descriptor units
-      auto issue_s = [&](int t, int j) {
-        const uint32_t klo = dk0.lo + (j % C::STAGES) * STAGE16;
+      auto issue_s = [&](int t, int g) {  // g: key tile counted over the CTA's items
+        const uint32_t klo = dk0.lo + (g % C::STAGES) * STAGE16;
         const uint32_t qlo = t ? dq1.lo : dq0.lo;
         const uint32_t dcol = tmem + (t ? C::COL_S1 : C::COL_S0);
 #pragma unroll
@@ -226,11 +274,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
         umma_commit(bar_s_full(t));
       };
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t vlo = dv0.lo + (j % C::STAGES) * STAGE16;
+      auto issue_pv = [&](int t, int g, bool acc) {
+        const uint32_t vlo = dv0.lo + (g % C::STAGES) * STAGE16;
         const uint32_t pcol = tmem + (t ? C::COL_S1 : C::COL_S0);
         const uint32_t ocol = tmem + (t ? C::COL_O1 : C::COL_O0);
-        const uint32_t acc0 = j > 0 ? 1u : 0u;
+        const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k) {
           // V: MN-major (d contiguous), 16 keys = 2 swizzle atoms of 8 rows. P of
@@ -239,51 +287,77 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                    k > 0 ? 1u : acc0);
         }
       };
-      bool ok = mbar_wait(bar_q, 0, abort_flag, 0x201) &&
-                mbar_wait(bar_kv_full(0), 0, abort_flag, 0x202);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-      }
-      int kv_waited = 0;  // highest key tile whose kv_full has been waited for
-      auto wait_kv = [&](int j) -> bool {
-        if (j <= kv_waited) return true;
-        kv_waited = j;
-        if (!mbar_wait(bar_kv_full(j % C::STAGES), (j / C::STAGES) & 1, abort_flag, 0x203)) return false;
+      bool ok = true;
+      int kg = 0;             // key tiles consumed so far (K/V ring position)
+      int jt0 = 0, jt1 = 0;   // key tiles of query tile 0 / 1 so far (s_full, p_full phases)
+      int kv_waited = -1;     // highest key tile (counted like kg) whose kv_full was waited for
+      auto wait_kv = [&](int g) -> bool {
+        if (g <= kv_waited) return true;
+        kv_waited = g;
+        if (!mbar_wait(bar_kv_full(g % C::STAGES), (g / C::STAGES) & 1, abort_flag, 0x203)) return false;
         tc_fence_after();
         return true;
       };
-      for (int j = 0; j < n1 && ok; ++j) {
-        if (j < n0) {
-          ok = mbar_wait(bar_p_full(0), j & 1, abort_flag, 0x204);
-          if (!ok) break;
-          FA2_TRACE_AT(trace_cta, 16, j);
-          tc_fence_after();
-          issue_pv(0, j);
-          if (j + 1 < n0) {
-            ok = wait_kv(j + 1);
+      for (int n = 0; ok; ++n) {
+        const int item = take_item(n, 0x207);
+        if (item < 0) break;
+        int pair, bh, n0, n1;
+        fwd_decode_item(item, p.n_pairs, p.BH, C::HEAD_GROUP, p.causal != 0, pair, bh);
+        tiles_of(pair, n0, n1);
+        FA2_TRACE_AT(trace_cta, 20, n);
+        ok = mbar_wait(bar_q_full, n & 1, abort_flag, 0x201) && wait_kv(kg);
+        if (!ok) break;
+        FA2_TRACE_AT(trace_cta, 21, n);
+        tc_fence_after();
+        // S of the item's first key tile: the S columns were last read by the
+        // previous item's PV, which this thread issued before
+        issue_s(0, kg);
+        issue_s(1, kg);
+        if (n1 == 1) umma_commit(bar_q_empty);  // every S of the item issued
+        for (int j = 0; j < n1 && ok; ++j) {
+          const int g = kg + j;
+          if (j < n0) {
+            ok = mbar_wait(bar_p_full(0), (jt0 + j) & 1, abort_flag, 0x204);
             if (!ok) break;
-            issue_s(0, j + 1);  // overwrites S0/P0 after PV0_j in issue order
-            FA2_TRACE_AT(trace_cta, 17, j);
+            if (j == 0 && n > 0) {  // the epilogue of the previous item has read O0
+              ok = mbar_wait(bar_o_free(0), (n - 1) & 1, abort_flag, 0x208);
+              if (!ok) break;
+            }
+            FA2_TRACE_AT(trace_cta && n == 0, 16, j);
+            tc_fence_after();
+            issue_pv(0, g, j > 0);
+            if (j + 1 < n0) {
+              ok = wait_kv(g + 1);
+              if (!ok) break;
+              issue_s(0, g + 1);  // overwrites S0/P0 after PV0 in issue order
+              FA2_TRACE_AT(trace_cta && n == 0, 17, j);
+            } else {
+              umma_commit(bar_o_done(0));
+            }
+          }
+          ok = mbar_wait(bar_p_full(1), (jt1 + j) & 1, abort_flag, 0x205);
+          if (!ok) break;
+          if (j == 0 && n > 0) {
+            ok = mbar_wait(bar_o_free(1), (n - 1) & 1, abort_flag, 0x209);
+            if (!ok) break;
+          }
+          FA2_TRACE_AT(trace_cta && n == 0, 18, j);
+          tc_fence_after();
+          issue_pv(1, g, j > 0);
+          umma_commit(bar_kv_empty(g % C::STAGES));  // K and V of this key tile fully consumed
+          if (j + 1 < n1) {
+            ok = wait_kv(g + 1);
+            if (!ok) break;
+            issue_s(1, g + 1);
+            if (j + 2 == n1) umma_commit(bar_q_empty);  // the item's last S: Q no longer read
+            FA2_TRACE_AT(trace_cta && n == 0, 19, j);
           } else {
-            umma_commit(bar_o_done(0));
+            umma_commit(bar_o_done(1));
           }
         }
-        ok = mbar_wait(bar_p_full(1), j & 1, abort_flag, 0x205);
-        if (!ok) break;
-        FA2_TRACE_AT(trace_cta, 18, j);
-        tc_fence_after();
-        issue_pv(1, j);
-        umma_commit(bar_kv_empty(j % C::STAGES));  // K_j and V_j fully consumed
-        if (j + 1 < n1) {
-          ok = wait_kv(j + 1);
-          if (!ok) break;
-          issue_s(1, j + 1);
-          FA2_TRACE_AT(trace_cta, 19, j);
-        } else {
-          umma_commit(bar_o_done(1));
-        }
+        kg += n1;
+        jt0 += n0;
+        jt1 += n1;
       }
       // drain: every UMMA of this CTA has finished before TMEM is released
       umma_commit(bar_drain);
@@ -294,9 +368,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int t = warp >> 3;              // query tile of this warpgroup
     const int h = (warp >> 2) & 1;        // key half: keys [64h, 64h+64) of each tile
     const int row = threadIdx.x & 127;    // TMEM lane
-    const int qt = t ? qt1 : qt0;
-    const int n_t = t ? n1 : n0;
-    const int qrow = qt * C::BM + row;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t scol = (t ? C::COL_S1 : C::COL_S0) + 64 * h;  // this half's scores
     constexpr int DH = D / 2;                                    // O columns per half
@@ -304,149 +375,169 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX) + t * 512 + row;  // + slot*256 + half*128
     float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM) + t * 512 + row;  // + half*256 + which*128
     const float c = p.scale_log2;
-    float m = -INFINITY;  // reference max of c * s, base-2 units (same in both halves)
-    float l = 0.f;        // this half's row sum of the weights 2^(c s - m)
-    float lr = 0.f;       // the same sum over the weights rounded to bf16
     bool ok = true;
+    int jt = 0;  // key tiles of this query tile over the CTA's items so far
+    for (int n = 0; ok; ++n) {
+      const int item = take_item(n, 0x306);
+      if (item < 0) break;
+      int pair, bh, n0, n1;
+      fwd_decode_item(item, p.n_pairs, p.BH, C::HEAD_GROUP, p.causal != 0, pair, bh);
+      tiles_of(pair, n0, n1);
+      const int qt = 2 * pair + t;
+      const int n_t = t ? n1 : n0;
+      const int qrow = qt * C::BM + row;
+      float m = -INFINITY;  // reference max of c * s, base-2 units (same in both halves)
+      float l = 0.f;        // this half's row sum of the weights 2^(c s - m)
+      float lr = 0.f;       // the same sum over the weights rounded to bf16
 #ifdef FA2_TRACE
-    const bool trace_row = trace_cta && row == 0 && h == 0;
+      const bool trace_row = trace_cta && n == 0 && row == 0 && h == 0;
+      const bool trace_item = trace_cta && row == 0 && h == 0;
 #endif
-    for (int j = 0; j < n_t; ++j) {
-      FA2_TRACE_AT(trace_row, 8 * t + 0, j);
-      ok = mbar_wait(bar_s_full(t), j & 1, abort_flag, 0x301);
-      if (!ok) break;
-      FA2_TRACE_AT(trace_row, 8 * t + 1, j);
-      tc_fence_after();
-      const int k0 = j * C::BN + 64 * h;  // first key of this half
-      const bool need_mask = (p.causal && j == qt) || (j * C::BN + C::BN > p.N);
-      const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys [0, lim) allowed
-      float s[64];
-      tmem_ld64(lane_base + scol, s);
-      if (need_mask) {
+      FA2_TRACE_AT(trace_item, 24 + 4 * t, n);
+      for (int j = 0; j < n_t; ++j) {
+        const int jj = jt + j;
+        FA2_TRACE_AT(trace_row, 8 * t + 0, j);
+        ok = mbar_wait(bar_s_full(t), jj & 1, abort_flag, 0x301);
+        if (!ok) break;
+        FA2_TRACE_AT(trace_row, 8 * t + 1, j);
+        FA2_TRACE_AT(trace_item && j == 0, 25 + 4 * t, n);
+        tc_fence_after();
+        const int k0 = j * C::BN + 64 * h;  // first key of this half
+        const bool need_mask = (p.causal && j == qt) || (j * C::BN + C::BN > p.N);
+        const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys [0, lim) allowed
+        float s[64];
+        tmem_ld64(lane_base + scol, s);
+        if (need_mask) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (k0 + i >= lim) s[i] = -INFINITY;
-      }
-      float mx;
-      {
-        float a = s[0], b = s[1];
-#pragma unroll
-        for (int i = 2; i < 62; i += 4) {
-          a = max3(a, s[i], s[i + 1]);
-          b = max3(b, s[i + 2], s[i + 3]);
+          for (int i = 0; i < 64; ++i)
+            if (k0 + i >= lim) s[i] = -INFINITY;
         }
-        mx = max3(a, b, fmaxf(s[62], s[63]));
-      }
-      // row max over both halves: publish this half's, read the other's
-      const int slot = j & 1;
-      xmax[slot * 256 + h * 128] = mx;
-      mbar_arrive(bar_xmax(t, slot));
-      ok = mbar_wait(bar_xmax(t, slot), (j >> 1) & 1, abort_flag, 0x304);
-      if (!ok) break;
-      mx = fmaxf(mx, xmax[slot * 256 + (1 - h) * 128]);
-      FA2_TRACE_AT(trace_row, 8 * t + 2, j);
-      const float m_cand = fmaxf(m, mx * c);
-      const bool grow = m_cand - m > C::RESCALE_THRESHOLD;  // always true for the first tile
-      const float alpha = grow ? ex2(m - m_cand) : 1.f;
-      if (grow) m = m_cand;
-      // weights 2^(c s - m) in pairs, written back over this half's S as bf16 P.
-      // rs: sum of the fp32 weights (for LSE); rr: sum of the bf16-rounded weights
-      // that the P V product actually uses (for O / l, so O stays a convex
-      // combination of V rows even when one weight dominates)
-      const unsigned long long c2 = f2(c, c), negm2 = f2(-m, -m);
-      unsigned long long rs2 = f2(0.f, 0.f), rr2 = f2(0.f, 0.f);
+        float mx;
+        {
+          float a = s[0], b = s[1];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t pk[16];
-        if (!need_mask) {
+          for (int i = 2; i < 62; i += 4) {
+            a = max3(a, s[i], s[i + 1]);
+            b = max3(b, s[i + 2], s[i + 3]);
+          }
+          mx = max3(a, b, fmaxf(s[62], s[63]));
+        }
+        // row max over both halves: publish this half's, read the other's
+        const int slot = jj & 1;
+        xmax[slot * 256 + h * 128] = mx;
+        mbar_arrive(bar_xmax(t, slot));
+        ok = mbar_wait(bar_xmax(t, slot), (jj >> 1) & 1, abort_flag, 0x304);
+        if (!ok) break;
+        mx = fmaxf(mx, xmax[slot * 256 + (1 - h) * 128]);
+        FA2_TRACE_AT(trace_row, 8 * t + 2, j);
+        const float m_cand = fmaxf(m, mx * c);
+        const bool grow = m_cand - m > C::RESCALE_THRESHOLD;  // always true for the first tile
+        const float alpha = grow ? ex2(m - m_cand) : 1.f;
+        if (grow) m = m_cand;
+        // weights 2^(c s - m) in pairs, written back over this half's S as bf16 P.
+        // rs: sum of the fp32 weights (for LSE); rr: sum of the bf16-rounded weights
+        // that the P V product actually uses (for O / l, so O stays a convex
+        // combination of V rows even when one weight dominates)
+        const unsigned long long c2 = f2(c, c), negm2 = f2(-m, -m);
+        unsigned long long rs2 = f2(0.f, 0.f), rr2 = f2(0.f, 0.f);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = 32 * q + 2 * i;
-            float x0, x1, p0, p1;
-            f2_split(f2_fma(f2(s[e], s[e + 1]), c2, negm2), x0, x1);
-            if ((16 * q + i) % C::POLY_EVERY == C::POLY_EVERY - 1) {
-              exp2_poly2(x0, x1, p0, p1);  // FMA pipe: balances the MUFU unit
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
+        for (int q = 0; q < 2; ++q) {
+          uint32_t pk[16];
+          if (!need_mask) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int e = 32 * q + 2 * i;
+              float x0, x1, p0, p1;
+              f2_split(f2_fma(f2(s[e], s[e + 1]), c2, negm2), x0, x1);
+              if ((16 * q + i) % C::POLY_EVERY == C::POLY_EVERY - 1) {
+                exp2_poly2(x0, x1, p0, p1);  // FMA pipe: balances the MUFU unit
+              } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              const uint32_t w = pack_bf16(p0, p1);
+              pk[i] = w;
+              rs2 = f2_add(rs2, f2(p0, p1));
+              rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
             }
-            const uint32_t w = pack_bf16(p0, p1);
-            pk[i] = w;
-            rs2 = f2_add(rs2, f2(p0, p1));
-            rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
-          }
-        } else {
-          // masked keys contribute exactly 0 (also when c == 0, where -inf * c is NaN)
+          } else {
+            // masked keys contribute exactly 0 (also when c == 0, where -inf * c is NaN)
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = 32 * q + 2 * i;
-            const float p0 = k0 + e >= lim ? 0.f : ex2(fmaf(s[e], c, -m));
-            const float p1 = k0 + e + 1 >= lim ? 0.f : ex2(fmaf(s[e + 1], c, -m));
-            const uint32_t w = pack_bf16(p0, p1);
-            pk[i] = w;
-            rs2 = f2_add(rs2, f2(p0, p1));
-            rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+            for (int i = 0; i < 16; ++i) {
+              const int e = 32 * q + 2 * i;
+              const float p0 = k0 + e >= lim ? 0.f : ex2(fmaf(s[e], c, -m));
+              const float p1 = k0 + e + 1 >= lim ? 0.f : ex2(fmaf(s[e + 1], c, -m));
+              const uint32_t w = pack_bf16(p0, p1);
+              pk[i] = w;
+              rs2 = f2_add(rs2, f2(p0, p1));
+              rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+            }
           }
+          // P of keys [32q, 32q+32) of this half -> columns [16q, 16q+16): the scores
+          // there are already in registers
+          tmem_st16(lane_base + scol + 16 * q, pk);
         }
-        // P of keys [32q, 32q+32) of this half -> columns [16q, 16q+16): the scores
-        // there are already in registers
-        tmem_st16(lane_base + scol + 16 * q, pk);
-      }
-      FA2_TRACE_AT(trace_row, 8 * t + 3, j);
-      float rs_lo, rs_hi, rr_lo, rr_hi;
-      f2_split(rs2, rs_lo, rs_hi);
-      f2_split(rr2, rr_lo, rr_hi);
-      l = l * alpha + (rs_lo + rs_hi);
-      lr = lr * alpha + (rr_lo + rr_hi);
-      // O holds PV_0..PV_{j-1}: all complete, since S_j was issued after them.
-      // Each half rescales its own D/2 columns of O.
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        FA2_TRACE_AT(trace_row, 8 * t + 3, j);
+        float rs_lo, rs_hi, rr_lo, rr_hi;
+        f2_split(rs2, rs_lo, rs_hi);
+        f2_split(rr2, rr_lo, rr_hi);
+        l = l * alpha + (rs_lo + rs_hi);
+        lr = lr * alpha + (rr_lo + rr_hi);
+        // O holds PV_0..PV_{j-1}: all complete, since S_j was issued after them.
+        // Each half rescales its own D/2 columns of O.
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-        for (int q = 0; q < DH / 32; ++q) {
-          float o[32];
-          tmem_ld32(lane_base + ocol + 32 * q, o);
-          uint32_t u[32];
+          for (int q = 0; q < DH / 32; ++q) {
+            float o[32];
+            tmem_ld32(lane_base + ocol + 32 * q, o);
+            uint32_t u[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(o[i] * alpha);
-          tmem_st32(lane_base + ocol + 32 * q, u);
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(o[i] * alpha);
+            tmem_st32(lane_base + ocol + 32 * q, u);
+          }
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p_full(t));
+        FA2_TRACE_AT(trace_row, 8 * t + 4, j);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p_full(t));
-      FA2_TRACE_AT(trace_row, 8 * t + 4, j);
-    }
-    if (ok && n_t > 0) ok = mbar_wait(bar_o_done(t), 0, abort_flag, 0x303);
-    if (ok) {
-      // row sums over both halves
+      if (!ok) break;
+      jt += n_t;
+      // epilogue: O / l. The row sums over both halves are exchanged while the
+      // item's last PV of this tile may still run.
       xsum[h * 256] = l;
       xsum[h * 256 + 128] = lr;
       mbar_arrive(bar_xsum(t));
-      ok = mbar_wait(bar_xsum(t), 0, abort_flag, 0x305);
-    }
-    if (ok) {
+      ok = mbar_wait(bar_xsum(t), n & 1, abort_flag, 0x305);
+      if (!ok) break;
       l += xsum[(1 - h) * 256];
       lr += xsum[(1 - h) * 256 + 128];
-      tc_fence_after();
       const float inv_l = 1.f / lr;
-      const bool store = qrow < p.N;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + qrow) * D + DH * h;
-#pragma unroll 1
+      ok = mbar_wait(bar_o_done(t), n & 1, abort_flag, 0x303);
+      if (!ok) break;
+      FA2_TRACE_AT(trace_item, 26 + 4 * t, n);
+      tc_fence_after();
+      // this half's D/2 columns, normalised and rounded to bf16 chunk by chunk
+      uint4 w[DH / 8];
+      uint32_t* wu = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
       for (int q = 0; q < DH / 32; ++q) {
-        float o[32];
-        tmem_ld32(lane_base + ocol + 32 * q, o);
-        uint4 w[4];
-        uint32_t* wu = reinterpret_cast<uint32_t*>(w);
+        float part[32];
+        tmem_ld32(lane_base + ocol + 32 * q, part);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) wu[i] = pack_bf16(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = w[i];
-        }
+        for (int i = 0; i < 16; ++i) wu[16 * q + i] = pack_bf16(part[2 * i] * inv_l, part[2 * i + 1] * inv_l);
       }
-      if (store && h == 0)
+      // O has been read: the next item's first PV may overwrite it
+      tc_fence_before();
+      mbar_arrive(bar_o_free(t));
+      {
+        const int row0 = qt * C::BM + (warp & 3) * 32;  // query row of lane 0
+        char* base = reinterpret_cast<char*>(p.o + (static_cast<size_t>(bh) * p.N + row0) * D + DH * h);
+        store_rows_coalesced<DH / 8>(base, static_cast<size_t>(D) * 2, w, __ballot_sync(0xffffffffu, qrow < p.N));
+      }
+      if (qrow < p.N && h == 0)
         p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * 0.69314718055994530942f;
+      FA2_TRACE_AT(trace_item, 27 + 4 * t, n);
     }
   }
 

@@ -163,6 +163,45 @@ __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Stores one row segment of G 16-byte chunks per lane, lane l's segment at
+// row0 + l * row_stride (bytes). Rows live on lanes (one TMEM lane each), so a
+// plain store of chunk c by every lane would touch 32 rows per instruction. An
+// xor-butterfly transposes the chunks inside each group of G lanes first: then
+// lane l holds chunk (l mod G) of the G rows of its group, and each store
+// instruction writes 32 / G whole segments of 16 G contiguous bytes.
+// Bit l of row_mask says whether lane l's row is stored.
+template <int G>
+__device__ __forceinline__ void store_rows_coalesced(char* row0, size_t row_stride, uint4 (&w)[G],
+                                                     unsigned int row_mask) {
+  static_assert(G == 2 || G == 4 || G == 8, "group of 2, 4 or 8 lanes");
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int b = 1; b < G; b <<= 1) {
+    const bool upper = (lane & b) != 0;
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      if (j & b) continue;
+      // the lower lane of the pair gives away chunk j|b, the upper lane chunk j
+      const uint4 x = upper ? w[j] : w[j | b];
+      uint4 y;
+      y.x = __shfl_xor_sync(0xffffffffu, x.x, b);
+      y.y = __shfl_xor_sync(0xffffffffu, x.y, b);
+      y.z = __shfl_xor_sync(0xffffffffu, x.z, b);
+      y.w = __shfl_xor_sync(0xffffffffu, x.w, b);
+      if (upper)
+        w[j] = y;
+      else
+        w[j | b] = y;
+    }
+  }
+  const int i = lane % G;
+  const int g0 = lane - i;
+#pragma unroll
+  for (int k = 0; k < G; ++k)
+    if ((row_mask >> (g0 + k)) & 1u)
+      *reinterpret_cast<uint4*>(row0 + static_cast<size_t>(g0 + k) * row_stride + i * 16) = w[k];
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (UMMA/TMA).
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

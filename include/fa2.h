@@ -64,7 +64,14 @@ typedef enum {
  * Forward pass: o = softmax(scale * q k^T [causal]) v and lse (natural log).
  * q, k, v: inputs [B,H,N,d] bf16. o: output [B,H,N,d] bf16. lse: output
  * [B,H,N] fp32, kept for the backward pass. causal: 0 or 1 (j <= i allowed).
- * One kernel launch on `stream`; the grid runs over (query block, batch*head).
+ * Work: pairs of 128-row query blocks x batch*head, taken from a work counter by
+ * a persistent grid of one CTA per SM. Enqueues on `stream` a 4-byte
+ * cudaMemsetAsync of that counter (one of 256 counters inside the library, used
+ * in turn) and one kernel launch. Launches that may overlap on the GPU (other
+ * streams) stay independent as long as fewer than 256 are in flight at once;
+ * launches ordered on one stream always are. The first call on a device looks
+ * up the counters' device address (cudaGetSymbolAddress): make it outside
+ * stream capture.
  */
 FA2_API fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse,
                        int B, int H, int N, int d, int causal, float scale, void* stream);
