@@ -461,12 +461,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
             }
           } else {
-            // masked keys contribute exactly 0 (also when c == 0, where -inf * c is NaN)
+            // masked keys get exponent -inf, hence weight exactly 0 (also when
+            // c == 0, where the masked score -inf times c is NaN)
+            const int nvalid = lim - k0;  // keys [k0, k0 + nvalid) of this half allowed
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int e = 32 * q + 2 * i;
-              const float p0 = k0 + e >= lim ? 0.f : ex2(fmaf(s[e], c, -m));
-              const float p1 = k0 + e + 1 >= lim ? 0.f : ex2(fmaf(s[e + 1], c, -m));
+              float x0, x1;
+              f2_split(f2_fma(f2(s[e], s[e + 1]), c2, negm2), x0, x1);
+              const float p0 = ex2(e < nvalid ? x0 : -INFINITY);
+              const float p1 = ex2(e + 1 < nvalid ? x1 : -INFINITY);
               const uint32_t w = pack_bf16(p0, p1);
               pk[i] = w;
               rs2 = f2_add(rs2, f2(p0, p1));
