@@ -167,8 +167,9 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
   // kv_full, kv_empty, st_full[S], st_empty[S], s_full, dp_full, p_ready,
   // ds_ready, dsm_free, dq_full, dq_empty, dkv_done, dkv_free, drain,
-  // item_full[2], item_empty[2], do_full[DS], do_empty[DS], staged, stg_free
-  static constexpr int NUM_BARS = 2 + 2 * STAGES + 10 + 4 + 2 * DO_STAGES + 2;
+  // item_full[2], item_empty[2], do_full[DS], do_empty[DS], staged, stg_free,
+  // epi_staged, dsbuf_free, epi_go
+  static constexpr int NUM_BARS = 2 + 2 * STAGES + 10 + 4 + 2 * DO_STAGES + 5;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;         // tmem slot, abort, items[2]
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   // d = 128 uses 231,6xx bytes: there is no room for alignment slack, so the
@@ -251,12 +252,14 @@ __device__ __forceinline__ void decode_item(int item, int n_ktiles, int BH, int 
 
 // WITH_DQ = false is the dK/dV-only variant used when dQ comes from the
 // separate query-parallel kernel (fa2_bwd_dq_kernel). tm_dq maps the fp32 dQ
-// accumulator for the TMA reductions.
+// accumulator for the TMA reductions, tm_dk / tm_dv the bf16 outputs for the
+// TMA stores of the epilogue.
 template <int D, bool WITH_DQ>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                   const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (C::NEEDS_ALIGNED_BASE && (smem_u32(smem_raw) & 1023u) != 0) {
@@ -293,6 +296,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   auto bar_do_empty = [&](int s) { return bar_s_full + 112 + 8 * (C::DO_STAGES + s); };
   const uint32_t bar_staged = bar_s_full + 112 + 16 * C::DO_STAGES;
   const uint32_t bar_stg_free = bar_staged + 8;
+  const uint32_t bar_epi_staged = bar_staged + 16;
+  const uint32_t bar_dsbuf_free = bar_staged + 24;
+  const uint32_t bar_epi_go = bar_staged + 32;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* item_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
@@ -326,6 +332,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     mbar_init(bar_staged, C::STG_THREADS);
     mbar_init(bar_stg_free, 1);
+    mbar_init(bar_epi_staged, C::ELEM_THREADS);
+    mbar_init(bar_dsbuf_free, 1);
+    mbar_init(bar_epi_go, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -339,6 +348,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_do);
     prefetch_tensormap(&tm_dq);
+    prefetch_tensormap(&tm_dk);
+    prefetch_tensormap(&tm_dv);
   }
   tc_fence_before();
   __syncthreads();
@@ -458,9 +469,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         int ktile, bh;
         decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
         const int n_iter = steps_of(ktile);
+        FA2_TRACE_AT(trace_cta, 40, n);
         ok = mbar_wait(bar_kv_full, n & 1, abort_flag, 0x1201) &&
              mbar_wait(bar_st_full(gs % C::STAGES), (gs / C::STAGES) & 1, abort_flag, 0x1202);
         if (!ok) break;
+        FA2_TRACE_AT(trace_cta, 41, n);
         tc_fence_after();
         // S^T of the item's first step: the elementwise warps read the previous
         // S^T before its p_ready, and its P^T is read by a dV issued earlier
@@ -550,11 +563,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_wait(bar_drain, 0, abort_flag, 0x1207);
     }
   } else if (warp == C::WARP_RED) {
-    // ---------------------------------------------------------- dQ reductions
-    // Once the staging threads have written d columns [0, 64) of step g's dQ
-    // tile to the staging buffer, one thread has the TMA add it into the fp32
-    // accumulator and frees the buffer as soon as the TMA has read it.
-    if (lane == 0 && WITH_DQ) {
+    // -------------------------------------------- dQ reductions, dK/dV stores
+    // Step g's staged dQ tile (d columns [0, 64)) is added into the fp32
+    // accumulator by TMA reductions; at the end of an item, dV (staged in the
+    // dS^T buffer) and scale * dK (in the staging buffer) go out by TMA stores.
+    // Each buffer is freed as soon as the TMA has read it. The staging buffer's
+    // uses (one per step, then one per item) are counted in this same order by
+    // the threads that stage dQ (stg_free); epi_go, one phase per item, tells
+    // every elementwise thread that the item's dQ tiles have been read.
+    if (lane == 0) {
       bool ok = true;
       int gs = 0;
       for (int n = 0; ok; ++n) {
@@ -564,7 +581,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
         const int i_first = p.causal ? ktile : 0;
         const int n_iter = steps_of(ktile);
-        for (int it = 0; it < n_iter; ++it) {
+        for (int it = 0; WITH_DQ && it < n_iter; ++it) {
           const int g = gs + it;
           ok = mbar_wait(bar_staged, g & 1, abort_flag, 0x1701);
           if (!ok) break;
@@ -574,12 +591,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           bulk_wait_group_read0();
           mbar_arrive(bar_stg_free);
         }
+        if (!ok) break;
+        mbar_arrive(bar_epi_go);
+        ok = mbar_wait(bar_epi_staged, n & 1, abort_flag, 0x1702);
+        if (!ok) break;
+        for (int c = 0; c < C::CHUNKS; ++c) {  // rows past N are not written by the TMA
+          tma_store_3d(&tm_dv, sbase + C::OFF_DS + c * C::CHUNK_BYTES, c * 64, ktile * C::BN, bh);
+          tma_store_3d(&tm_dk, sbase + C::OFF_STG + c * C::CHUNK_BYTES, c * 64, ktile * C::BN, bh);
+        }
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(bar_dsbuf_free);
+        mbar_arrive(bar_stg_free);
         gs += n_iter;
       }
-      bulk_wait_group0();  // every reduction has landed before the kernel ends
-    } else if (lane == 0) {
-      for (int n = 0;; ++n)  // dK/dV only: take part in the item hand-off, nothing else
-        if (take_item(n, 0x1709) < 0) break;
+      bulk_wait_group0();  // every reduction and store has landed before the kernel ends
     }
   } else {
     // ------------------------------------------------ elementwise groups (0-15)
@@ -598,6 +624,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
       const int i_first = p.causal ? ktile : 0;
       const int n_iter = steps_of(ktile);
+      FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 44, n);
 #ifdef FA2_TRACE
       // group 0: a thread of the first warp (dQ staging at d = 128); group 1: a
       // thread of the third warp (dQ reductions at d = 128)
@@ -622,8 +649,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           mbar_arrive(bar_dq_empty);
           if (r < 64) {
             // staged: row q of box r/32 holds query CW g + q; d = r sits in 16-byte
-            // unit ((r mod 32) / 4) xor (row mod 8) of the 128-byte swizzle
-            if (gg > 0 && !mbar_wait(bar_stg_free, (gg - 1) & 1, abort_flag, 0x1306)) return false;
+            // unit ((r mod 32) / 4) xor (row mod 8) of the 128-byte swizzle. This is
+            // staging-buffer use gg + n: every earlier step and item epilogue used it.
+            if (gg + n > 0 && !mbar_wait(bar_stg_free, (gg + n - 1) & 1, abort_flag, 0x1306)) return false;
             const uint32_t box = stg + (r >> 5) * C::STG_BOX_BYTES;
             const uint32_t unit = static_cast<uint32_t>((r & 31) >> 2);
             const uint32_t word = static_cast<uint32_t>(r & 3) * 4;
@@ -648,7 +676,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           tmem_ld16(lane_base + C::COL_DQ + DW * g, v);
           tc_fence_before();
           mbar_arrive(bar_dq_empty);
-          if (gg > 0 && !mbar_wait(bar_stg_free, (gg - 1) & 1, abort_flag, 0x1306)) return false;
+          if (gg + n > 0 && !mbar_wait(bar_stg_free, (gg + n - 1) & 1, abort_flag, 0x1306)) return false;
 #pragma unroll
           for (int u = 0; u < DW / 4; ++u) {
             const int col = DW * g + 4 * u;
@@ -676,6 +704,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         ok = mbar_wait(bar_s_full, gg & 1, abort_flag, 0x1301);
         if (!ok) break;
         FA2_TRACE_AT(trace_row, 8 * g + 1, it);
+        FA2_TRACE_AT(trace_cta && threadIdx.x == 0 && it == 0, 43, n);
         tc_fence_after();
         // P^T for query columns [CW g, CW g + CW)
         uint32_t pk[CW / 2];
@@ -735,7 +764,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             dk[e / 2 + 1] = pack_bf16(s2, s3);
           }
         }
-        if (gg > 0) {  // dK and dQ of the previous step have finished reading the dS^T tile
+        if (it == 0 && n > 0) {  // the TMA has read the previous item's dV staged there
+          ok = mbar_wait(bar_dsbuf_free, (n - 1) & 1, abort_flag, 0x1307);
+          if (!ok) break;
+        } else if (gg > 0) {  // dK and dQ of the previous step have finished reading the dS^T tile
           ok = mbar_wait(bar_dsm_free, (gg - 1) & 1, abort_flag, 0x1303);
           if (!ok) break;
         }
@@ -750,19 +782,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         FA2_TRACE_AT(trace_row, 8 * g + 3, it);
       }
       if (WITH_DQ && ok) ok = drain(n_iter - 1);
+      FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 45, n);
       if (ok) ok = mbar_wait(bar_dkv_done, n & 1, abort_flag, 0x1305);
 #ifdef FA2_TRACE
       FA2_TRACE_AT(trace_row, 32, 0);
+      FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 46, n);
 #endif
       if (!ok) break;
-      // epilogue: group g stores d columns [g D/4, (g+1) D/4) of dV and scale * dK;
-      // the TMEM columns are released before the stores
+      // epilogue: group g stages d columns [g D/4, (g+1) D/4) of dV (in the dS^T
+      // buffer: the item's last dK and dQ MMAs are done) and of scale * dK (in the
+      // staging buffer, once the TMA has read its last dQ tile), 128-byte-swizzled
+      // like the tensor maps; the reduction warp stores them with the TMA. The
+      // TMEM columns are released first.
       {
         constexpr int DW = D / C::NWG;
         tc_fence_after();
-        const int key = ktile * C::BN + r;
-        const bool store = key < p.N;
-        const size_t off = (static_cast<size_t>(bh) * p.N + key) * D + DW * g;
         float v[DW], w[DW];
         if constexpr (DW == 32) {
           tmem_ld32(lane_base + C::COL_DV + DW * g, v);
@@ -773,19 +807,31 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
         tc_fence_before();
         mbar_arrive(bar_dkv_free);
-        // rows on lanes: transposed in groups of lanes so that every store
-        // instruction writes whole 2*DW-byte row segments
-        const unsigned int rows = __ballot_sync(0xffffffffu, store);
-        const size_t off0 = off - static_cast<size_t>(r & 31) * D;  // lane 0's row
-        uint4 o[DW / 8];
-        uint32_t* ou = reinterpret_cast<uint32_t*>(o);
+        uint32_t pk[DW / 2];
 #pragma unroll
-        for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-        store_rows_coalesced<DW / 8>(reinterpret_cast<char*>(p.dv + off0), static_cast<size_t>(D) * 2, o, rows);
+        for (int e = 0; e < DW / 2; ++e) pk[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
 #pragma unroll
-        for (int e = 0; e < DW / 2; ++e) ou[e] = pack_bf16(w[2 * e] * p.scale, w[2 * e + 1] * p.scale);
-        store_rows_coalesced<DW / 8>(reinterpret_cast<char*>(p.dk + off0), static_cast<size_t>(D) * 2, o, rows);
+        for (int u = 0; u < DW / 8; ++u) {
+          const uint32_t off = sw128_offset(r, (DW / 8) * g + u);
+          *reinterpret_cast<uint4*>(smem + C::OFF_DS + off) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+#pragma unroll
+        for (int e = 0; e < DW / 2; ++e) pk[e] = pack_bf16(w[2 * e] * p.scale, w[2 * e + 1] * p.scale);
+        // the TMA has read every dQ tile of this item from the staging buffer (and,
+        // before those, the previous item's dK)
+        ok = mbar_wait(bar_epi_go, n & 1, abort_flag, 0x1308);
+        if (!ok) break;
+#pragma unroll
+        for (int u = 0; u < DW / 8; ++u) {
+          const uint32_t off = sw128_offset(r, (DW / 8) * g + u);
+          *reinterpret_cast<uint4*>(smem + C::OFF_STG + off) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        fence_async_smem();
+        mbar_arrive(bar_epi_staged);
       }
+      FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 47, n);
       gs += n_iter;
     }
   }

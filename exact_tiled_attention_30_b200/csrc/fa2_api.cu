@@ -266,10 +266,11 @@ fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const vo
     if (st != FA2_OK) return st;
   }
   const WsLayout w = ws_layout(workspace, BH, N, D);
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
   if (!make_map_bhnd(&tq, q, BH, N, D, 128) || !make_map_bhnd(&tk, k, BH, N, D, 128) ||
       !make_map_bhnd(&tv, v, BH, N, D, 128) || !make_map_bhnd(&tdo, dO, BH, N, D, 128) ||
-      !make_map_acc(&tdq, w.dq_acc, BH, w.Np, D))
+      !make_map_acc(&tdq, w.dq_acc, BH, w.Np, D) || !make_map_bhnd(&tdk, dk, BH, N, D, 128) ||
+      !make_map_bhnd(&tdv, dv, BH, N, D, 128))
     return FA2_ERR_CUDA;
   fa2::BwdParams bp;
   bp.dk = reinterpret_cast<__nv_bfloat16*>(dk);
@@ -288,7 +289,8 @@ fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const vo
   // persistent: one CTA per SM (its shared memory allows no second one)
   const long long items = static_cast<long long>(bp.n_ktiles) * BH;
   const int ctas = static_cast<int>(items < sm_count(dev) ? items : sm_count(dev));
-  fa2::fa2_bwd_kernel<D, WITH_DQ><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, tdq, bp);
+  fa2::fa2_bwd_kernel<D, WITH_DQ><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, tdo, tdq, tdk,
+                                                                                    tdv, bp);
   return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
 
