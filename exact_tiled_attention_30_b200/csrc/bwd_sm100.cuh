@@ -35,21 +35,19 @@ struct BwdPreParams {
   unsigned int* counter;  // work-item counter of the main kernel
   int N;
   int Np;
-  long long rows;  // BH * Np
 };
 
-// 16 threads per row (d = 128) or 8 (d = 64), 16 bytes of O and dO per thread.
+// Grid (row blocks, batch*head). 16 threads per row (d = 128) or 8 (d = 64),
+// 16 bytes of O and dO per thread.
 template <int D>
 __global__ void __launch_bounds__(256) fa2_bwd_pre_kernel(const BwdPreParams p) {
   constexpr int TPR = D / 8;            // threads per row
   constexpr int RPB = 256 / TPR;        // rows per block per sweep
   const int sub = threadIdx.x % TPR;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.counter = 0u;
-  const long long stride = static_cast<long long>(gridDim.x) * RPB;
-  for (long long r = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / TPR; r < p.rows;
-       r += stride) {
-    const long long bh = r / p.Np;
-    const int n = static_cast<int>(r - bh * p.Np);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.counter = 0u;
+  const long long bh = blockIdx.y;
+  for (int n = blockIdx.x * RPB + threadIdx.x / TPR; n < p.Np; n += gridDim.x * RPB) {
+    const long long r = bh * p.Np + n;  // row of the [BH][Np] workspace arrays
     float acc = 0.f;
     if (n < p.N) {
       const size_t off = (static_cast<size_t>(bh) * p.N + n) * D + sub * 8;
@@ -85,21 +83,19 @@ struct BwdConvertParams {
   int N;
   int Np;
   int d;
-  long long total8;     // BH * N * d / 8
+  int head8;            // N * d / 8: groups of 8 elements per head
   float scale;
 };
 
+// Grid (element blocks, batch*head). Within a head the accumulator and dQ are
+// both row-major with row stride d (the accumulator's padding rows come last),
+// so element e of the head is at offset e in both.
 __global__ void __launch_bounds__(256) fa2_bwd_dq_convert_kernel(const BwdConvertParams p) {
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  const int per_row8 = p.d / 8;
-  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < p.total8;
-       t += stride) {
-    const long long row = t / per_row8;  // bh * N + n
-    const int c8 = static_cast<int>(t - row * per_row8);
-    const long long bh = row / p.N;
-    const long long n = row - bh * p.N;
-    const float4* src =
-        reinterpret_cast<const float4*>(p.dq_acc + (static_cast<size_t>(bh) * p.Np + n) * p.d + c8 * 8);
+  const size_t bh = blockIdx.y;
+  const float* src_head = p.dq_acc + bh * p.Np * p.d;
+  __nv_bfloat16* dst_head = p.dq + bh * p.N * p.d;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < p.head8; t += gridDim.x * blockDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(src_head + static_cast<size_t>(t) * 8);
     const float4 a = src[0];
     const float4 b = src[1];
     uint4 w;
@@ -107,7 +103,7 @@ __global__ void __launch_bounds__(256) fa2_bwd_dq_convert_kernel(const BwdConver
     w.y = pack_bf16(a.z * p.scale, a.w * p.scale);
     w.z = pack_bf16(b.x * p.scale, b.y * p.scale);
     w.w = pack_bf16(b.z * p.scale, b.w * p.scale);
-    *reinterpret_cast<uint4*>(p.dq + static_cast<size_t>(row) * p.d + c8 * 8) = w;
+    *reinterpret_cast<uint4*>(dst_head + static_cast<size_t>(t) * 8) = w;
   }
 }
 

@@ -229,8 +229,13 @@ int sm_count(int dev) {
   return count[dev];
 }
 
-inline int grid_cap(long long want) {
-  return static_cast<int>(want < 148LL * 16 ? (want > 0 ? want : 1) : 148LL * 16);
+// Grid (blocks per head, heads) of the streaming kernels: about 16 blocks per SM
+// in total, each looping over its share of a head.
+inline dim3 per_head_grid(long long want_per_head, int BH) {
+  long long x = (148LL * 16 + BH - 1) / BH;
+  if (x > want_per_head) x = want_per_head;
+  if (x < 1) x = 1;
+  return dim3(static_cast<unsigned int>(x), static_cast<unsigned int>(BH));
 }
 
 template <int D>
@@ -247,9 +252,8 @@ fa2_status launch_bwd_pre(const void* o, const float* lse, const void* dO, int B
   pp.counter = w.counter;
   pp.N = N;
   pp.Np = w.Np;
-  pp.rows = static_cast<long long>(BH) * w.Np;
   constexpr int rpb = 256 / (D / 8);
-  fa2::fa2_bwd_pre_kernel<D><<<grid_cap((pp.rows + rpb - 1) / rpb), 256, 0, stream>>>(pp);
+  fa2::fa2_bwd_pre_kernel<D><<<per_head_grid((w.Np + rpb - 1) / rpb, BH), 256, 0, stream>>>(pp);
   return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
 
@@ -337,9 +341,9 @@ fa2_status launch_bwd_convert(void* dq, int BH, int N, int d, float scale, void*
   cp.N = N;
   cp.Np = w.Np;
   cp.d = d;
-  cp.total8 = static_cast<long long>(BH) * N * d / 8;
+  cp.head8 = N * (d / 8);
   cp.scale = scale;
-  fa2::fa2_bwd_dq_convert_kernel<<<grid_cap((cp.total8 + 255) / 256), 256, 0, stream>>>(cp);
+  fa2::fa2_bwd_dq_convert_kernel<<<per_head_grid((cp.head8 + 255) / 256, BH), 256, 0, stream>>>(cp);
   return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
 
