@@ -525,11 +525,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           if (!ok) break;
           FA2_TRACE_AT(trace_cta && n == 0, 19, it);
           tc_fence_after();
-          const uint32_t qmlo = dQm.lo + s * TILE16;
+          auto issue_dk = [&]() {
+            const uint32_t qmlo = dQm.lo + s * TILE16;
 #pragma unroll
-          for (int k = 0; k < C::BM / 16; ++k)
-            umma_ss2(tmem + C::COL_DK, dSk.lo + kmaj(k), dSk.hi, qmlo + k * (2048 >> 4), dQm.hi,
-                     IDESC_KV, k > 0 ? 1u : acc0);
+            for (int k = 0; k < C::BM / 16; ++k)
+              umma_ss2(tmem + C::COL_DK, dSk.lo + kmaj(k), dSk.hi, qmlo + k * (2048 >> 4), dQm.hi,
+                       IDESC_KV, k > 0 ? 1u : acc0);
+          };
+          // d = 128 issues dQ first: its drain gates the next step's dP, which
+          // reuses its TMEM columns (measured +1-4 %; d = 64, -2 %, keeps dK first)
+          if (!C::DQ_IN_DP) issue_dk();
           if constexpr (WITH_DQ) {
             if (!C::DQ_IN_DP && g > 0) {  // dQ of step g-1 must be read out before it is overwritten
               ok = mbar_wait(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1206);
@@ -547,6 +552,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             }
             umma_commit(bar_dq_full);
           }
+          if (C::DQ_IN_DP) issue_dk();
           umma_commit(bar_dsm_free);
           umma_commit(bar_st_empty(s));
         }
