@@ -356,3 +356,42 @@ def attention_forward_backward_host(q, k, v, dout, causal: bool = False, scale: 
     fa2_forward_backward_host(q, k, v, dout, o, lse, dq, dk, dv, causal, scale, workspace,
                               heads_per_chunk, stream)
     return o, lse, dq, dk, dv
+
+
+def _autograd_function():
+    import torch
+
+    class _Attention(torch.autograd.Function):
+        """Exact attention with both passes on the C ABI (fa2_forward, fa2_backward)."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, causal, scale):
+            o, lse = attention_forward(q, k, v, causal=causal, scale=scale)
+            ctx.save_for_backward(q, k, v, o, lse)
+            ctx.causal, ctx.scale = causal, scale
+            return o
+
+        @staticmethod
+        def backward(ctx, dout):
+            q, k, v, o, lse = ctx.saved_tensors
+            dq, dk, dv = attention_backward(q, k, v, o, lse, dout.contiguous(), causal=ctx.causal,
+                                            scale=ctx.scale)
+            return dq, dk, dv, None, None
+
+    return _Attention
+
+
+_ATTENTION_FN = None
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None):
+    """softmax(scale * q k^T [causal]) v as a differentiable PyTorch op: the forward
+    and backward passes run in this library's kernels (q, k, v: contiguous bf16
+    CUDA tensors [B, H, N, d]; d in {64, 128}). The drop-in form of the method
+    for code that trains through attention with autograd."""
+    global _ATTENTION_FN
+    if _ATTENTION_FN is None:
+        _ATTENTION_FN = _autograd_function()
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    return _ATTENTION_FN.apply(q, k, v, bool(causal), float(scale))

@@ -121,3 +121,31 @@ def test_forward_repeatable(fa2, d, causal):
     for _ in range(20):
         o, lse = fa2.attention_forward(q, k, v, causal=causal)
         assert torch.equal(o, o0) and torch.equal(lse, l0)
+
+
+def test_forward_work_counters(fa2):
+    """Each forward launch takes the next of the library's 256 work counters: 300
+    launches in a row (the ring wraps) and launches on two streams at once must
+    give the same bits as a single launch."""
+    import torch
+
+    t = gh.inputs(34, 2, 3, 384, 64)
+    q, k, v = (gh.to_device(t[n]) for n in ("q", "k", "v"))
+    scale = 0.125
+    o_ref, lse_ref = fa2.attention_forward(q, k, v, causal=True, scale=scale)
+    o, lse = torch.empty_like(o_ref), torch.empty_like(lse_ref)
+    for _ in range(300):
+        fa2.fa2_forward(q, k, v, o, lse, True, scale)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    outs = [(torch.empty_like(o_ref), torch.empty_like(lse_ref)) for _ in range(2)]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for _ in range(20):
+        for s, (oo, ll) in zip(streams, outs):
+            fa2.fa2_forward(q, k, v, oo, ll, True, scale, s)
+    torch.cuda.synchronize()
+    for oo, ll in outs:
+        assert torch.equal(oo, o_ref) and torch.equal(ll, lse_ref)
+    st, site = fa2.fa2_get_device_status()
+    assert st == 0, f"device status {fa2.fa2_status_string(st)} at site {site:#x}"
