@@ -55,6 +55,16 @@ def _bind(lib):
                                                    ctypes.c_double, pi64, i64, pi64, i64,
                                                    d, d, d, ctypes.c_int]
     lib.oracle_attention_backward_rows.restype = ctypes.c_int
+    lib.oracle_attention_forward_qk.argtypes = [d, d, d, i64, i64, i64, i64, ctypes.c_int,
+                                                ctypes.c_double, pi64, i64, d, d, ctypes.c_int]
+    lib.oracle_attention_forward_qk.restype = ctypes.c_int
+    lib.oracle_attention_backward_qk.argtypes = [d, d, d, d, i64, i64, i64, i64, ctypes.c_int,
+                                                 ctypes.c_double, d, d, d, d, d, ctypes.c_int]
+    lib.oracle_attention_backward_qk.restype = ctypes.c_int
+    lib.oracle_attention_backward_rows_qk.argtypes = [d, d, d, d, i64, i64, i64, i64, ctypes.c_int,
+                                                      ctypes.c_double, pi64, i64, pi64, i64,
+                                                      d, d, d, ctypes.c_int]
+    lib.oracle_attention_backward_rows_qk.restype = ctypes.c_int
     lib.oracle_default_threads.restype = ctypes.c_int
     return lib
 
@@ -117,14 +127,17 @@ def _heads(x: np.ndarray):
 
 
 def attention_forward(q, k, v, causal: bool, scale: float, rows=None, nthreads: int = 0):
-    """O and LSE of standard attention. q, k, v: [..., N, d] (fp64 or bf16 bits).
+    """O and LSE of standard attention. q: [..., Nq, d], k, v: [..., Nk, d] (fp64 or
+    bf16 bits); causal masking is aligned to the bottom-right corner (query i sees
+    keys j <= i + Nk - Nq).
 
-    Returns (o [..., R, d], lse [..., R]) with R = len(rows) or N.
+    Returns (o [..., R, d], lse [..., R]) with R = len(rows) or Nq.
     """
     qh, lead = _heads(q)
     kh, _ = _heads(k)
     vh, _ = _heads(v)
     nh, N, d = qh.shape
+    Nk = kh.shape[1]
     if rows is None:
         rp, R = None, N
     else:
@@ -132,29 +145,34 @@ def attention_forward(q, k, v, causal: bool, scale: float, rows=None, nthreads: 
         rp, R = _ptr(rows_a, ctypes.c_int64), rows_a.size
     o = np.empty((nh, R, d))
     lse = np.empty((nh, R))
-    rc = _active().oracle_attention_forward(_ptr(qh), _ptr(kh), _ptr(vh), nh, N, d, int(causal),
-                                          float(scale), rp, R, _ptr(o), _ptr(lse), int(nthreads))
+    rc = _active().oracle_attention_forward_qk(_ptr(qh), _ptr(kh), _ptr(vh), nh, N, Nk, d,
+                                             int(causal), float(scale), rp, R, _ptr(o), _ptr(lse),
+                                             int(nthreads))
     if rc != 0:
         raise ValueError("oracle_attention_forward rejected its arguments")
     return o.reshape(*lead, R, d), lse.reshape(*lead, R)
 
 
 def attention_backward(q, k, v, dout, causal: bool, scale: float, nthreads: int = 0):
-    """Full backward. Returns dict with o, lse, dq, dk, dv (fp64, input shapes)."""
+    """Full backward. Returns dict with o, lse, dq, dk, dv (fp64; o, lse, dq shaped
+    like q, dk and dv like k)."""
     qh, lead = _heads(q)
     kh, _ = _heads(k)
     vh, _ = _heads(v)
     dh, _ = _heads(dout)
     nh, N, d = qh.shape
-    out = {name: np.empty((nh, N, d)) for name in ("o", "dq", "dk", "dv")}
+    Nk = kh.shape[1]
+    out = {name: np.empty((nh, N, d)) for name in ("o", "dq")}
+    out.update({name: np.empty((nh, Nk, d)) for name in ("dk", "dv")})
     out["lse"] = np.empty((nh, N))
-    rc = _active().oracle_attention_backward(_ptr(qh), _ptr(kh), _ptr(vh), _ptr(dh), nh, N, d,
-                                           int(causal), float(scale), _ptr(out["o"]),
-                                           _ptr(out["lse"]), _ptr(out["dq"]), _ptr(out["dk"]),
-                                           _ptr(out["dv"]), int(nthreads))
+    rc = _active().oracle_attention_backward_qk(_ptr(qh), _ptr(kh), _ptr(vh), _ptr(dh), nh, N, Nk,
+                                              d, int(causal), float(scale), _ptr(out["o"]),
+                                              _ptr(out["lse"]), _ptr(out["dq"]), _ptr(out["dk"]),
+                                              _ptr(out["dv"]), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_attention_backward rejected its arguments")
-    res = {name: a.reshape(*lead, N, d) for name, a in out.items() if name != "lse"}
+    res = {name: out[name].reshape(*lead, N, d) for name in ("o", "dq")}
+    res.update({name: out[name].reshape(*lead, Nk, d) for name in ("dk", "dv")})
     res["lse"] = out["lse"].reshape(*lead, N)
     return res
 
@@ -170,13 +188,14 @@ def attention_backward_rows(q, k, v, dout, causal: bool, scale: float, qrows, kr
     vh, _ = _heads(v)
     dh, _ = _heads(dout)
     nh, N, d = qh.shape
+    Nk = kh.shape[1]
     qr = np.ascontiguousarray(qrows, dtype=np.int64)
     kr = np.ascontiguousarray(krows, dtype=np.int64)
     dq = np.empty((nh, qr.size, d))
     dk = np.empty((nh, kr.size, d))
     dv = np.empty((nh, kr.size, d))
-    rc = _active().oracle_attention_backward_rows(
-        _ptr(qh), _ptr(kh), _ptr(vh), _ptr(dh), nh, N, d, int(causal), float(scale),
+    rc = _active().oracle_attention_backward_rows_qk(
+        _ptr(qh), _ptr(kh), _ptr(vh), _ptr(dh), nh, N, Nk, d, int(causal), float(scale),
         _ptr(qr, ctypes.c_int64), qr.size, _ptr(kr, ctypes.c_int64), kr.size,
         _ptr(dq), _ptr(dk), _ptr(dv), int(nthreads))
     if rc != 0:

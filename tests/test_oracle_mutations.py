@@ -14,15 +14,17 @@ import pytest
 
 import oracle
 from tests import test_oracle as pins
+from tests import test_oracle_qk as pins_qk
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.cpp")
 
 MUTANTS = {
     "ds_sign": ("dsi[j] = pi[j] * (dp[j] - D[(size_t)i]);", "dsi[j] = pi[j] * (dp[j] + D[(size_t)i]);"),
     "dq_drops_scale": ("dqh[i * d + c] *= scale;", "dqh[i * d + c] *= 1.0;"),
-    "dk_transposed_ds": ("const double ds = dS[(size_t)(i * N + j)];",
-                         "const double ds = dS[(size_t)(j * N + i)];"),
-    "causal_off_by_one": ("return causal ? i + 1 : N;", "return causal ? std::min(i + 2, N) : N;"),
+    "dk_transposed_ds": ("const double ds = dS[(size_t)(i * Nk + j)];",
+                         "const double ds = dS[(size_t)(j * Nk + i)];"),
+    "causal_off_by_one": ("return causal ? std::min(Nk, i + 1 + Nk - Nq) : Nk;",
+                          "return causal ? std::min(Nk, i + 2 + Nk - Nq) : Nk;"),
     "lse_drops_max": ("return m + std::log(l);", "return std::log(l);"),
     "dv_uses_ds": ("dvj[c] += p * doi[c];", "dvj[c] += ds * doi[c];"),
     "scores_drop_scale": ("for (int64_t j = j0; j < j1; ++j) acc[j - j0] *= scale;", ""),
@@ -30,9 +32,11 @@ MUTANTS = {
                  "D[(size_t)i] = dot(doh + i * d, vh + i * d, d);"),
     "rows_p_drops_lse": ("ds[j] = std::exp(s[j] - L[(size_t)i]) * (dp[j] - D[(size_t)i]);",
                          "ds[j] = std::exp(s[j]) * (dp[j] - D[(size_t)i]);"),
-    "rows_dk_drops_scale": ("      for (int64_t c = 0; c < d; ++c) dkj[c] *= scale;\n    });\n  }\n  return 0;\n}\n\nint oracle_default",
-                            "    });\n  }\n  return 0;\n}\n\nint oracle_default"),
+    "rows_dk_drops_scale": ("      for (int64_t c = 0; c < d; ++c) dkj[c] *= scale;\n    });\n  }\n  return 0;\n}\n\nint oracle_attention_backward_rows(",
+                            "    });\n  }\n  return 0;\n}\n\nint oracle_attention_backward_rows("),
     "pv_transposed": ("const double* r = rows + j * d;", "const double* r = rows + j;"),
+    "causal_top_left": ("return causal ? std::min(Nk, i + 1 + Nk - Nq) : Nk;",
+                        "return causal ? std::min(Nk, i + 1) : Nk;"),
 }
 
 
@@ -47,6 +51,10 @@ def _run_pins():
     pins.test_causal_row_zero(oracle)
     pins.test_shift_invariance(oracle)
     pins.test_single_token(oracle)
+    # different query and key lengths (bottom-right causal alignment)
+    pins_qk.test_brute_force(oracle, 3, 7, 4, True)
+    pins_qk.test_brute_force(oracle, 7, 3, 4, False)
+    pins_qk.test_uniform_scores_bottom_right(oracle)
 
 
 def test_pins_pass_on_the_committed_oracle():
