@@ -77,6 +77,11 @@ def load_library():
     lib.fa2_backward_main_dkdv.restype = i
     lib.fa2_backward_dq.argtypes = [vp] * 5 + [i, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t, vp]
     lib.fa2_backward_dq.restype = i
+    lib.fa2_forward_qk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float, vp]
+    lib.fa2_forward_qk.restype = i
+    lib.fa2_backward_qk.argtypes = [vp] * 9 + [i, i, i, i, i, i, ctypes.c_float, vp, ctypes.c_size_t,
+                                              vp]
+    lib.fa2_backward_qk.restype = i
     lib.fa2_forward_backward_host_workspace_size.argtypes = [i, i, i, i, i]
     lib.fa2_forward_backward_host_workspace_size.restype = ctypes.c_size_t
     lib.fa2_forward_backward_host.argtypes = [vp] * 9 + [i, i, i, i, i, ctypes.c_float, i, vp,
@@ -250,8 +255,50 @@ def fa2_clear_device_status() -> None:
     _check("fa2_clear_device_status", load_library().fa2_clear_device_status())
 
 
+def fa2_forward_qk(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """C ABI fa2_forward_qk: q, o [B,H,Nq,d], k, v [B,H,Nk,d] bf16; lse fp32 [B,H,Nq].
+    Causal masking is aligned to the bottom-right corner (query i sees keys
+    j <= i + Nk - Nq)."""
+    import torch
+
+    B, H, Nq, d = _bhnd(q)
+    Nk = int(k.shape[2])
+    for t, n, rows in ((q, "q", Nq), (k, "k", Nk), (v, "v", Nk), (o, "o", Nq)):
+        _require(t, n, torch.bfloat16)
+        if tuple(t.shape) != (B, H, rows, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, rows, d)}")
+    _require(lse, "lse", torch.float32)
+    if tuple(lse.shape) != (B, H, Nq):
+        raise ValueError("lse must be [B, H, Nq]")
+    _check("fa2_forward_qk", load_library().fa2_forward_qk(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, int(bool(causal)),
+        float(scale), _stream(stream)))
+
+
+def fa2_backward_qk(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float, workspace,
+                    stream=None) -> None:
+    """C ABI fa2_backward_qk (shapes as fa2_forward_qk; dq like q, dk and dv like k;
+    workspace of fa2_backward_workspace_size(B, H, Nq, d) bytes)."""
+    import torch
+
+    B, H, Nq, d = _bhnd(q)
+    Nk = int(k.shape[2])
+    for t, n, rows in ((q, "q", Nq), (k, "k", Nk), (v, "v", Nk), (o, "o", Nq), (dout, "dout", Nq),
+                       (dq, "dq", Nq), (dk, "dk", Nk), (dv, "dv", Nk)):
+        _require(t, n, torch.bfloat16)
+        if tuple(t.shape) != (B, H, rows, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, rows, d)}")
+    _require(lse, "lse", torch.float32)
+    _require(workspace, "workspace")
+    _check("fa2_backward_qk", load_library().fa2_backward_qk(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, H, Nq, Nk, d, int(bool(causal)), float(scale), _ptr(workspace), _nbytes(workspace),
+        _stream(stream)))
+
+
 def attention_forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
-    """Allocates o and lse, runs fa2_forward, returns (o, lse)."""
+    """Allocates o and lse, runs fa2_forward (fa2_forward_qk when k and q differ in
+    length), returns (o, lse)."""
     import torch
 
     B, H, N, d = _bhnd(q)
@@ -259,7 +306,10 @@ def attention_forward(q, k, v, causal: bool = False, scale: float | None = None,
         scale = d ** -0.5
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    fa2_forward(q, k, v, o, lse, causal, scale, stream)
+    if k.shape[2] != N:
+        fa2_forward_qk(q, k, v, o, lse, causal, scale, stream)
+    else:
+        fa2_forward(q, k, v, o, lse, causal, scale, stream)
     return o, lse
 
 
@@ -275,7 +325,11 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: float
     if workspace is None:
         workspace = torch.empty(fa2_backward_workspace_size(B, H, N, d), dtype=torch.uint8,
                                 device=q.device)
-    fa2_backward_ex(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, dq_strategy, stream)
+    if k.shape[2] != N:  # different key length: fa2_backward_qk (dQ by reductions)
+        fa2_backward_qk(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, stream)
+    else:
+        fa2_backward_ex(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, dq_strategy,
+                        stream)
     return dq, dk, dv
 
 

@@ -201,20 +201,15 @@ struct BwdParams {
   const float* lse2;      // [BH][Np]
   const float* delta;     // [BH][Np]
   unsigned int* counter;  // next work item (zeroed by the preprocess kernel)
-  int N;
-  int Np;
+  int Np;                 // query rows rounded up to 128
   int BH;
-  int n_ktiles;
+  int n_ktiles;           // key tiles: ceil(Nk / 128)
+  int n_qtiles;           // query tiles: Np / 128
+  int kq_offset;          // Nk - Nq: causal query i sees keys j <= i + kq_offset
   int causal;
   float scale;
   float scale_log2;
 };
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
 
 __device__ __forceinline__ void red_add(float* addr, float a) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
@@ -360,7 +355,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_arrive(bar_item_empty(n & 1));
     return item;
   };
-  auto steps_of = [&](int ktile) { return p.causal ? p.n_ktiles - ktile : p.n_ktiles; };
+  // causal: the first query tile that sees key tile ktile (query i sees keys
+  // j <= i + kq_offset, the mask aligned to the bottom-right corner)
+  auto qfirst = [&](int ktile) {
+    const int x = ktile * C::BN - p.kq_offset;
+    return p.causal && x > 0 ? x / C::BM : 0;
+  };
+  auto steps_of = [&](int ktile) { return p.n_qtiles - qfirst(ktile); };
 
   if (warp == C::WARP_TMA) {
     // --------------------------------------------------- scheduler + TMA producer
@@ -382,7 +383,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (item < 0) break;
         int ktile, bh;
         decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
-        const int i_first = p.causal ? ktile : 0;
+        const int i_first = qfirst(ktile);
         const int n_iter = steps_of(ktile);
         for (int it = 0; it < n_iter && ok; ++it, ++gs) {
           const int i = i_first + it;
@@ -581,7 +582,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (item < 0) break;
         int ktile, bh;
         decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
-        const int i_first = p.causal ? ktile : 0;
+        const int i_first = qfirst(ktile);
         const int n_iter = steps_of(ktile);
         for (int it = 0; WITH_DQ && it < n_iter; ++it) {
           const int g = gs + it;
@@ -624,7 +625,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       if (item < 0) break;
       int ktile, bh;
       decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
-      const int i_first = p.causal ? ktile : 0;
+      const int i_first = qfirst(ktile);
       const int n_iter = steps_of(ktile);
       FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 44, n);
 #ifdef FA2_TRACE
@@ -714,7 +715,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           float sv[CW];
           tmem_ld32(lane_base + C::COL_S + CW * g, sv);
           const unsigned long long c2 = f2(c, c);
-          const bool diag = p.causal && (i == ktile);
+          // keys past query q + off are masked; off >= 127 masks none
+          const int off = i * C::BM + p.kq_offset - ktile * C::BN;
+          const bool diag = p.causal && off < C::BN - 1;
 #pragma unroll
           for (int e = 0; e < CW; e += 4) {
             const float4 l4 = *reinterpret_cast<const float4*>(lse2 + e);
@@ -722,12 +725,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
             f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
             float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-            if (diag) {  // query i*128 + q sees key k0 + r only if q >= r
+            if (diag) {  // query i*128 + q sees key ktile*128 + r only if r <= q + off
               const int q = CW * g + e;
-              if (q < r) p0 = 0.f;
-              if (q + 1 < r) p1 = 0.f;
-              if (q + 2 < r) p2 = 0.f;
-              if (q + 3 < r) p3 = 0.f;
+              if (q + off < r) p0 = 0.f;
+              if (q + 1 + off < r) p1 = 0.f;
+              if (q + 2 + off < r) p2 = 0.f;
+              if (q + 3 + off < r) p3 = 0.f;
             }
             pk[e / 2] = pack_bf16(p0, p1);
             pk[e / 2 + 1] = pack_bf16(p2, p3);

@@ -164,7 +164,8 @@ unsigned int* fwd_counter(int dev, cudaStream_t stream, fa2_status* st) {
 
 template <int D>
 fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                          int H, int N, int causal, float scale, cudaStream_t stream, int dev) {
+                          int H, int Nq, int Nk, int causal, float scale, cudaStream_t stream,
+                          int dev) {
   using C = FwdCfg<D>;
   static bool smem_set[kMaxDevices] = {false};
   static std::mutex mu;
@@ -175,14 +176,16 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   }
   const int BH = B * H;
   CUtensorMap tq, tk, tv;
-  if (!make_map_bhnd(&tq, q, BH, N, D, 128) || !make_map_bhnd(&tk, k, BH, N, D, 128) ||
-      !make_map_bhnd(&tv, v, BH, N, D, 128))
+  if (!make_map_bhnd(&tq, q, BH, Nq, D, 128) || !make_map_bhnd(&tk, k, BH, Nk, D, 128) ||
+      !make_map_bhnd(&tv, v, BH, Nk, D, 128))
     return FA2_ERR_CUDA;
   fa2::FwdParams p;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
-  p.N = N;
-  p.n_qtiles = (N + C::BM - 1) / C::BM;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.kq_offset = Nk - Nq;
+  p.n_qtiles = (Nq + C::BM - 1) / C::BM;
   p.n_pairs = (p.n_qtiles + 1) / 2;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -259,8 +262,8 @@ fa2_status launch_bwd_pre(const void* o, const float* lse, const void* dO, int B
 
 template <int D, bool WITH_DQ = true>
 fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk,
-                           void* dv, int BH, int N, int causal, float scale, void* workspace,
-                           cudaStream_t stream, int dev) {
+                           void* dv, int BH, int Nq, int Nk, int causal, float scale,
+                           void* workspace, cudaStream_t stream, int dev) {
   using C = fa2::BwdCfg<D>;
   static bool smem_set[kMaxDevices] = {false};
   static std::mutex mu;
@@ -269,12 +272,12 @@ fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const vo
     fa2_status st = ensure_smem(fa2::fa2_bwd_kernel<D, WITH_DQ>, C::SMEM_ALLOC, dev, smem_set);
     if (st != FA2_OK) return st;
   }
-  const WsLayout w = ws_layout(workspace, BH, N, D);
+  const WsLayout w = ws_layout(workspace, BH, Nq, D);
   CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
-  if (!make_map_bhnd(&tq, q, BH, N, D, 128) || !make_map_bhnd(&tk, k, BH, N, D, 128) ||
-      !make_map_bhnd(&tv, v, BH, N, D, 128) || !make_map_bhnd(&tdo, dO, BH, N, D, 128) ||
-      !make_map_acc(&tdq, w.dq_acc, BH, w.Np, D) || !make_map_bhnd(&tdk, dk, BH, N, D, 128) ||
-      !make_map_bhnd(&tdv, dv, BH, N, D, 128))
+  if (!make_map_bhnd(&tq, q, BH, Nq, D, 128) || !make_map_bhnd(&tk, k, BH, Nk, D, 128) ||
+      !make_map_bhnd(&tv, v, BH, Nk, D, 128) || !make_map_bhnd(&tdo, dO, BH, Nq, D, 128) ||
+      !make_map_acc(&tdq, w.dq_acc, BH, w.Np, D) || !make_map_bhnd(&tdk, dk, BH, Nk, D, 128) ||
+      !make_map_bhnd(&tdv, dv, BH, Nk, D, 128))
     return FA2_ERR_CUDA;
   fa2::BwdParams bp;
   bp.dk = reinterpret_cast<__nv_bfloat16*>(dk);
@@ -283,10 +286,11 @@ fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const vo
   bp.lse2 = w.lse2;
   bp.delta = w.delta;
   bp.counter = w.counter;
-  bp.N = N;
   bp.Np = w.Np;
   bp.BH = BH;
-  bp.n_ktiles = w.Np / 128;
+  bp.n_ktiles = (Nk + 127) / 128;
+  bp.n_qtiles = w.Np / 128;
+  bp.kq_offset = Nk - Nq;
   bp.causal = causal ? 1 : 0;
   bp.scale = scale;
   bp.scale_log2 = scale * 1.4426950408889634f;
@@ -347,6 +351,17 @@ fa2_status launch_bwd_convert(void* dq, int BH, int N, int d, float scale, void*
   return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
 
+// Query and key lengths of the _qk entry points: each within the limits of one
+// sequence, and causal only with Nq <= Nk (bottom-right alignment leaves no
+// query row without keys).
+fa2_status check_qk(int B, int H, int Nq, int Nk, int d, int causal, float scale) {
+  fa2_status st = check_common(B, H, Nq, d, scale);
+  if (st == FA2_OK) st = check_common(B, H, Nk, d, scale);
+  if (st != FA2_OK) return st;
+  if (causal && Nq > Nk) return FA2_ERR_UNSUPPORTED;
+  return FA2_OK;
+}
+
 fa2_status check_workspace(int B, int H, int N, int d, const void* workspace, size_t bytes) {
   if (!workspace) return FA2_ERR_INVALID_ARG;
   if (bytes < fa2_backward_workspace_size(B, H, N, d)) return FA2_ERR_INVALID_ARG;
@@ -381,8 +396,51 @@ fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, flo
   st = check_device(&dev);
   if (st != FA2_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_forward<64>(q, k, v, o, lse, B, H, N, causal, scale, s, dev);
-  return launch_forward<128>(q, k, v, o, lse, B, H, N, causal, scale, s, dev);
+  if (d == 64) return launch_forward<64>(q, k, v, o, lse, B, H, N, N, causal, scale, s, dev);
+  return launch_forward<128>(q, k, v, o, lse, B, H, N, N, causal, scale, s, dev);
+}
+
+fa2_status fa2_forward_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int H, int Nq, int Nk, int d, int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_qk(B, H, Nq, Nk, d, causal, scale);
+  if (st != FA2_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA2_ERR_MISALIGNED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_forward<64>(q, k, v, o, lse, B, H, Nq, Nk, causal, scale, s, dev);
+  return launch_forward<128>(q, k, v, o, lse, B, H, Nq, Nk, causal, scale, s, dev);
+}
+
+fa2_status fa2_backward_qk(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                           int H, int Nq, int Nk, int d, int causal, float scale, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA2_ERR_INVALID_ARG;
+  fa2_status st = check_qk(B, H, Nq, Nk, d, causal, scale);
+  if (st != FA2_OK) return st;
+  st = check_workspace(B, H, Nq, d, workspace, workspace_bytes);
+  if (st != FA2_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA2_ERR_MISALIGNED;
+  int dev = 0;
+  st = check_device(&dev);
+  if (st != FA2_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (d == 64) {
+    st = launch_bwd_pre<64>(o, lse, dO, BH, Nq, workspace, s);
+    if (st == FA2_OK) st = launch_bwd_main<64>(q, k, v, dO, dk, dv, BH, Nq, Nk, causal, scale, workspace, s, dev);
+  } else {
+    st = launch_bwd_pre<128>(o, lse, dO, BH, Nq, workspace, s);
+    if (st == FA2_OK) st = launch_bwd_main<128>(q, k, v, dO, dk, dv, BH, Nq, Nk, causal, scale, workspace, s, dev);
+  }
+  if (st == FA2_OK) st = launch_bwd_convert(dq, BH, Nq, d, scale, workspace, s);
+  return st;
 }
 
 size_t fa2_backward_workspace_size(int B, int H, int N, int d) {
@@ -424,8 +482,8 @@ fa2_status fa2_backward_main(const void* q, const void* k, const void* v, const 
   st = check_device(&dev);
   if (st != FA2_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd_main<64>(q, k, v, dO, dk, dv, B * H, N, causal, scale, workspace, s, dev)
-                 : launch_bwd_main<128>(q, k, v, dO, dk, dv, B * H, N, causal, scale, workspace, s, dev);
+  return d == 64 ? launch_bwd_main<64>(q, k, v, dO, dk, dv, B * H, N, N, causal, scale, workspace, s, dev)
+                 : launch_bwd_main<128>(q, k, v, dO, dk, dv, B * H, N, N, causal, scale, workspace, s, dev);
 }
 
 fa2_status fa2_backward_dq_convert(void* dq, int B, int H, int N, int d, float scale,
@@ -459,8 +517,8 @@ fa2_status fa2_backward_main_dkdv(const void* q, const void* k, const void* v, c
   if (st != FA2_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return d == 64
-             ? launch_bwd_main<64, false>(q, k, v, dO, dk, dv, B * H, N, causal, scale, workspace, s, dev)
-             : launch_bwd_main<128, false>(q, k, v, dO, dk, dv, B * H, N, causal, scale, workspace, s, dev);
+             ? launch_bwd_main<64, false>(q, k, v, dO, dk, dv, B * H, N, N, causal, scale, workspace, s, dev)
+             : launch_bwd_main<128, false>(q, k, v, dO, dk, dv, B * H, N, N, causal, scale, workspace, s, dev);
 }
 
 fa2_status fa2_backward_dq(const void* q, const void* k, const void* v, const void* dO, void* dq,
@@ -505,15 +563,15 @@ fa2_status fa2_backward_ex(const void* q, const void* k, const void* v, const vo
   if (d == 64) {
     st = launch_bwd_pre<64>(o, lse, dO, BH, N, workspace, s);
     if (st == FA2_OK)
-      st = separate ? launch_bwd_main<64, false>(q, k, v, dO, dk, dv, BH, N, causal, scale, workspace, s, dev)
-                    : launch_bwd_main<64, true>(q, k, v, dO, dk, dv, BH, N, causal, scale, workspace, s, dev);
+      st = separate ? launch_bwd_main<64, false>(q, k, v, dO, dk, dv, BH, N, N, causal, scale, workspace, s, dev)
+                    : launch_bwd_main<64, true>(q, k, v, dO, dk, dv, BH, N, N, causal, scale, workspace, s, dev);
     if (st == FA2_OK && separate)
       st = launch_bwd_dq<64>(q, k, v, dO, dq, BH, N, causal, scale, workspace, s, dev);
   } else {
     st = launch_bwd_pre<128>(o, lse, dO, BH, N, workspace, s);
     if (st == FA2_OK)
-      st = separate ? launch_bwd_main<128, false>(q, k, v, dO, dk, dv, BH, N, causal, scale, workspace, s, dev)
-                    : launch_bwd_main<128, true>(q, k, v, dO, dk, dv, BH, N, causal, scale, workspace, s, dev);
+      st = separate ? launch_bwd_main<128, false>(q, k, v, dO, dk, dv, BH, N, N, causal, scale, workspace, s, dev)
+                    : launch_bwd_main<128, true>(q, k, v, dO, dk, dv, BH, N, N, causal, scale, workspace, s, dev);
     if (st == FA2_OK && separate)
       st = launch_bwd_dq<128>(q, k, v, dO, dq, BH, N, causal, scale, workspace, s, dev);
   }
@@ -628,10 +686,10 @@ fa2_status fa2_backward_noalloc(const void* q, const void* k, const void* v, con
   // so whatever an earlier call left in the array does not matter
   if (d == 64) {
     st = launch_bwd_pre<64>(o, lse, dO, BH, N, scratch, s);
-    if (st == FA2_OK) st = launch_bwd_main<64>(q, k, v, dO, dk, dv, BH, N, causal, scale, scratch, s, dev);
+    if (st == FA2_OK) st = launch_bwd_main<64>(q, k, v, dO, dk, dv, BH, N, N, causal, scale, scratch, s, dev);
   } else {
     st = launch_bwd_pre<128>(o, lse, dO, BH, N, scratch, s);
-    if (st == FA2_OK) st = launch_bwd_main<128>(q, k, v, dO, dk, dv, BH, N, causal, scale, scratch, s, dev);
+    if (st == FA2_OK) st = launch_bwd_main<128>(q, k, v, dO, dk, dv, BH, N, N, causal, scale, scratch, s, dev);
   }
   if (st == FA2_OK) st = launch_bwd_convert(dq, BH, N, d, scale, scratch, s);
   return st;

@@ -85,8 +85,10 @@ struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   unsigned int* counter;  // next work item, zero at launch
-  int N;
-  int n_qtiles;  // ceil(N / 128)
+  int Nq;        // query rows (O, LSE)
+  int Nk;        // key rows
+  int kq_offset; // Nk - Nq: causal query i sees keys j <= i + kq_offset
+  int n_qtiles;  // ceil(Nq / 128)
   int n_pairs;   // ceil(n_qtiles / 2)
   int BH;
   int causal;
@@ -128,11 +130,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_items = p.n_pairs * p.BH;
-  const int n_kv_total = (p.N + C::BN - 1) / C::BN;
-  // query tiles 2*pair and 2*pair+1; with causal masking tile t sees key tiles [0, qt_t]
+  const int n_kv_total = (p.Nk + C::BN - 1) / C::BN;
+  // query tiles 2*pair and 2*pair+1; with causal masking the last row of tile qt
+  // sees keys up to qt*128 + 127 + kq_offset (self-attention: key tiles [0, qt])
   auto tiles_of = [&](int pair, int& n0, int& n1) {
-    n0 = p.causal ? min(n_kv_total, 2 * pair + 1) : n_kv_total;
-    n1 = p.causal ? min(n_kv_total, 2 * pair + 2) : n_kv_total;  // n1 >= n0
+    n0 = p.causal ? min(n_kv_total, (2 * pair * C::BM + C::BM - 1 + p.kq_offset) / C::BN + 1) : n_kv_total;
+    n1 = p.causal ? min(n_kv_total, ((2 * pair + 1) * C::BM + C::BM - 1 + p.kq_offset) / C::BN + 1)
+                  : n_kv_total;  // n0 <= n1 <= n0 + 1
   };
 #ifdef FA2_TRACE
   const bool trace_cta = blockIdx.x == 7;
@@ -403,8 +407,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         FA2_TRACE_AT(trace_item && j == 0, 25 + 4 * t, n);
         tc_fence_after();
         const int k0 = j * C::BN + 64 * h;  // first key of this half
-        const bool need_mask = (p.causal && j == qt) || (j * C::BN + C::BN > p.N);
-        const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys [0, lim) allowed
+        // some row of the tile has keys of this tile masked (causal limit or Nk)
+        const bool need_mask = (p.causal && j * C::BN + C::BN > qt * C::BM + 1 + p.kq_offset) ||
+                               (j * C::BN + C::BN > p.Nk);
+        const int lim = p.causal ? min(qrow + 1 + p.kq_offset, p.Nk) : p.Nk;  // keys [0, lim) allowed
         float s[64];
         tmem_ld64(lane_base + scol, s);
         if (need_mask) {
@@ -536,11 +542,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       mbar_arrive(bar_o_free(t));
       {
         const int row0 = qt * C::BM + (warp & 3) * 32;  // query row of lane 0
-        char* base = reinterpret_cast<char*>(p.o + (static_cast<size_t>(bh) * p.N + row0) * D + DH * h);
-        store_rows_coalesced<DH / 8>(base, static_cast<size_t>(D) * 2, w, __ballot_sync(0xffffffffu, qrow < p.N));
+        char* base = reinterpret_cast<char*>(p.o + (static_cast<size_t>(bh) * p.Nq + row0) * D + DH * h);
+        store_rows_coalesced<DH / 8>(base, static_cast<size_t>(D) * 2, w, __ballot_sync(0xffffffffu, qrow < p.Nq));
       }
-      if (qrow < p.N && h == 0)
-        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * 0.69314718055994530942f;
+      if (qrow < p.Nq && h == 0)
+        p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = (m + __log2f(l)) * 0.69314718055994530942f;
       FA2_TRACE_AT(trace_item, 27 + 4 * t, n);
     }
   }

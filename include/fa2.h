@@ -195,6 +195,26 @@ FA2_API fa2_status fa2_backward_noalloc(const void* q, const void* k, const void
                                         int causal, float scale, void* stream);
 
 /*
+ * Different query and key lengths (cross attention): q, o, dO, dq are
+ * [B, H, Nq, d], k, v, dk, dv [B, H, Nk, d], lse [B, H, Nq]; the workspace is
+ * fa2_backward_workspace_size(B, H, Nq, d) bytes. With causal = 1 the mask is
+ * aligned to the bottom-right corner of the Nq x Nk score matrix: query i sees
+ * keys j <= i + Nk - Nq (the pages only use Nq = Nk, where this is j <= i;
+ * the bottom-right reading is ours). Causal with Nq > Nk (rows without keys)
+ * returns FA2_ERR_UNSUPPORTED, like d not in {64, 128}. Otherwise the same
+ * arguments, checks, kernels and errors as fa2_forward / fa2_backward (the
+ * backward uses the dQ-reduction strategy); fa2_forward and fa2_backward are
+ * these with Nq = Nk = N.
+ */
+FA2_API fa2_status fa2_forward_qk(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                                  void* stream);
+FA2_API fa2_status fa2_backward_qk(const void* q, const void* k, const void* v, const void* o,
+                                   const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                   int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Forward and backward from HOST buffers: the form of the computation for
  * callers whose tensors live in host memory (and how end-to-end throughput,
  * host<->device copies included, is measured). The pages' method itself is the

@@ -178,3 +178,32 @@ def test_host_path_rejects_bad_arguments(lib):
     p = [A] * 10
     p[9] = A + 16  # the device workspace must be 256-byte aligned
     assert host(lib, p) == 3
+
+
+def test_qk_entry_points_reject_bad_arguments(lib):
+    f = ctypes.c_float
+
+    def fwd_qk(Nq=100, Nk=300, causal=1, d=64, p=None):
+        p = [A] * 5 if p is None else p
+        return lib.fa2_forward_qk(*p, 1, 2, Nq, Nk, d, causal, f(0.125), None)
+
+    assert fwd_qk(Nq=300, Nk=100, causal=1) == 2  # causal needs Nq <= Nk
+    assert fwd_qk(Nq=0) == 1 and fwd_qk(Nk=0) == 1
+    assert fwd_qk(d=80) == 2
+    assert fwd_qk(p=[A, None, A, A, A]) == 1
+    assert fwd_qk(p=[A, A + 8, A, A, A]) == 3
+    ws = lib.fa2_backward_workspace_size(1, 2, 100, 64)
+
+    def bwd_qk(Nq=100, Nk=300, causal=1, wsb=ws, p=None):
+        p = [A] * 10 if p is None else p
+        return lib.fa2_backward_qk(*p[:9], 1, 2, Nq, Nk, 64, causal, f(0.125), p[9], wsb, None)
+
+    assert bwd_qk(Nq=300, Nk=100, causal=1) == 2
+    assert bwd_qk(wsb=ws - 1) == 1
+    for i in range(10):
+        p = [A] * 10
+        p[i] = None
+        assert bwd_qk(p=p) == 1, i
+    p = [A] * 10
+    p[7] = A + 4
+    assert bwd_qk(p=p) == 3
