@@ -14,8 +14,8 @@
 //   1. fa2_bwd_pre: D and LSE * log2(e) into the workspace (rows padded to a
 //      multiple of 128: D = 0, LSE = +inf there so P vanishes), dQ accumulator
 //      and the main kernel's work-item counter zeroed. HBM-bound.
-//   2. fa2_bwd_kernel: one CTA per (128-key block, batch*head), parallel over key
-//      blocks; dK and dV accumulate in tensor memory over all query blocks, dQ
+//   2. fa2_bwd_kernel: persistent, parallel over (128-key block, batch*head)
+//      items; dK and dV accumulate in tensor memory over all query blocks, dQ
 //      is added into an fp32 accumulator with reductions (layout below).
 //   3. fa2_bwd_dq_convert: dQ = bf16(scale * accumulator).
 #pragma once
@@ -112,25 +112,32 @@ __global__ void __launch_bounds__(256) fa2_bwd_dq_convert_kernel(const BwdConver
 // Persistent: one CTA per SM takes work items (128-key block j, batch*head)
 // from a counter in the workspace, longest first within groups of heads
 // (causal: low j sees the most query blocks). Per item, query blocks i stream
-// through a two-stage TMA ring (causal: only i >= j, the diagonal block first).
+// through a two-stage TMA ring (causal: only the blocks that see block j, the
+// diagonal one first; with Nq != Nk query i sees keys <= i + Nk - Nq).
 //   warp 16       TMA producer and scheduler: fetches the next item, hands it to
 //                 the other warps through a two-slot ring, loads K_j, V_j once the
-//                 previous item's MMAs are done, then Q_i, dO_i, LSE2_i, D_i
+//                 previous item's MMAs are done, then Q_i with LSE2_i and D_i (two
+//                 stages) and dO_i (one buffer at d = 128, two at d = 64)
 //   warp 17       MMA issuer + TMEM owner, per step:
 //                   S^T = K Q_i^T,  dP^T = V dO_i^T          (keys on TMEM lanes)
 //                   dV += P^T dO_i    (P^T from TMEM)
 //                   dK += dS^T Q_i    (dS^T from smem, K-major)
 //                   d = 128: dQ^T = K^T dS^T (d on lanes; dS^T read MN-major)
 //                   d =  64: dQ   = dS K     (queries on lanes)
+//   warp 18       reductions and stores: adds each step's staged dQ tile into
+//                 the fp32 accumulator with TMA tensor reductions and, after an
+//                 item, writes its dK and dV with TMA tensor stores
 //   warps 0-15    four elementwise warpgroups; warpgroup g owns query columns
 //                 [32g, 32g + 32) of a step and thread r key row r. P^T =
 //                 exp2(c S^T - LSE2) goes back into TMEM over the group's own
 //                 S^T columns; dS^T = P^T (dP^T - D) goes to swizzled smem; then
-//                 the group adds its share of dQ into the fp32 accumulator with
-//                 reductions. No row statistics are needed (P comes from the
-//                 saved LSE), so the groups never exchange data. After an item's
-//                 last step they store dK, dV, while the MMA warp already starts
-//                 the next item.
+//                 the group's share of dQ goes to the fp32 accumulator: at
+//                 d = 128 rows d < 64 through the staging buffer and warp 18,
+//                 the rest with red.global; at d = 64 all through the staging
+//                 buffer. No row statistics are needed (P comes from the saved
+//                 LSE), so the groups never exchange data. After an item's last
+//                 step they stage dV and scale * dK for warp 18's stores, while
+//                 the MMA warp already starts the next item.
 // Tensor memory: S^T [0,128) (P^T of group g in [32g, 32g+16)), dP^T [128,256),
 // dV [256,256+D), dK [256+D,256+2D); dQ^T (d = 128) reuses the dP^T columns once
 // dS is in smem, dQ (d = 64) has [384,448).

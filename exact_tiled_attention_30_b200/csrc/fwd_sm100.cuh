@@ -3,16 +3,22 @@
 // Method ("FlashAttention-2" summary page, How It Works items 1-3; "FlashAttention
 // (v2)" glossary page, definition and mechanism paragraphs; reproduction page of
 // the FlashAttention-2 paper, closing paragraph on causal blocks):
-//   * the sequence is split across CTAs, not just batch and heads: one CTA per
-//     (256-row query block, batch*head);
+//   * the sequence is split across CTAs, not just batch and heads: the work
+//     items are (256-row query block, batch*head) pairs, taken by a persistent
+//     grid of one CTA per SM from a work counter, heaviest first;
 //   * K/V tiles of 128 keys stream through shared memory; the running row max m
 //     and row sum l (online softmax) keep the N x N scores on chip;
 //   * the accumulator is divided by l once, in the epilogue;
 //   * causal: key tiles wholly above the diagonal are never visited and only
-//     the diagonal tile of each query tile is masked elementwise.
+//     the diagonal tile of each query tile is masked elementwise (with Nq != Nk
+//     the diagonal is that of the bottom-right corner: query i sees keys
+//     j <= i + Nk - Nq).
 //
 // B200 mapping (the pages' A100/H100 tiling is prior art only):
-//   warp 16       TMA producer: Q0, Q1 once, then K_j/V_j into a STAGES-deep ring
+//   warp 16       scheduler + TMA producer: takes the next item, hands it to the
+//                 other warps through a two-slot ring, loads Q0, Q1 once the
+//                 previous item's last S MMA is done, K_j/V_j into a STAGES-deep
+//                 ring that continues across items
 //   warp 17       MMA issuer + TMEM owner. Per key tile j it issues
 //                 PV0_j, S0_{j+1}, PV1_j, S1_{j+1} (in that order), so while one
 //                 tile's softmax runs the tensor core works on the other tile:
@@ -27,7 +33,10 @@
 //                 shared memory, so both use one reference max), exp2, partial
 //                 row sums, P written back as bf16 over the first 32 of its S
 //                 columns. Halving the per-thread row shortens the softmax step
-//                 that sits between the two MMAs of a tile.
+//                 that sits between the two MMAs of a tile. Epilogue per item:
+//                 O / l, stored with lanes transposed in groups so that every
+//                 store instruction writes whole row segments; O is released to
+//                 the next item's first PV as soon as it has been read.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D). Scores are kept in base 2: c = scale * log2(e) folds the
 // softmax scale into the exponent and m is stored pre-multiplied by c.
