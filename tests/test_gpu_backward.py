@@ -188,3 +188,22 @@ def test_strategies_agree(fa2):
 
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
     assert gh.rel_fro(gh.to_host_f64(a[0]), gh.to_host_f64(b[0])) < 5e-3
+
+
+@pytest.mark.parametrize("N,d,causal", [(3, 64, True), (2, 128, False)])
+def test_maximum_head_count(fa2, oracle_mod, N, d, causal):
+    """B*H = 65535, the largest the library accepts (one grid dimension of the
+    streaming kernels; 65535 work items for each attention kernel): every head is
+    computed, checked on sampled heads. Short sequences keep the inputs small."""
+    import torch
+
+    B, H = 65535, 1
+    t = gh.inputs(47, B, H, N, d, with_do=True)
+    scale = 1.0 / math.sqrt(d)
+    got = run_fwd_bwd(fa2, t, causal, scale)
+    torch.cuda.synchronize()
+    for b, h in gh.sample_heads(B, H, 6, seed=N):
+        ref = oracle_mod.attention_backward(t["q"][b, h], t["k"][b, h], t["v"][b, h],
+                                            t["do"][b, h], causal, scale)
+        assert np.all(np.abs(got["o"][b, h] - ref["o"]) <= gh.o_tolerance(ref["o"]))
+        check_grads({n: got[n][b, h] for n in ("dq", "dk", "dv")}, ref, f"head ({b},{h})")
