@@ -271,6 +271,69 @@ def workload_config(args, w):
     }
 
 
+# ------------------------------------------------------- benchmark-figure grid
+def grid_points():
+    """The pages' attention benchmark axes: hidden size 2048 (H = 2048 / d),
+    d in {64, 128}, N in 512 .. 16k with B = 16384 / N, causal and not."""
+    pts = []
+    for d in (64, 128):
+        for causal in (False, True):
+            for N in (512, 1024, 2048, 4096, 8192, 16384):
+                pts.append({"B": 16384 // N, "H": 2048 // d, "N": N, "d": d, "causal": causal})
+    return pts
+
+
+def run_grid(args):
+    """One JSON line per grid point: forward, backward (three kernels) and their sum
+    in TFLOP/s on device-resident random bf16 inputs, CUDA events around `reps`
+    calls after warm-up (not the contract line; the contract line is the default
+    run)."""
+    import torch
+
+    import exact_tiled_attention_30_b200 as fa2
+
+    fa2.load_library()
+    peaks, _ = load_peaks()
+    reps = max(args.steps // 40, 5)
+    for w in grid_points():
+        B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+        scale = 1.0 / math.sqrt(d)
+        q = torch.randn(B, H, N, d, device="cuda", dtype=torch.bfloat16)
+        k, v, do = torch.randn_like(q), torch.randn_like(q), torch.randn_like(q)
+        o = torch.empty_like(q)
+        lse = torch.empty(B, H, N, device="cuda", dtype=torch.float32)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        ws = torch.empty(fa2.fa2_backward_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+
+        def fwd():
+            fa2.fa2_forward(q, k, v, o, lse, causal, scale)
+
+        def bwd():
+            fa2.fa2_backward(q, k, v, o, lse, do, dq, dk, dv, causal, scale, ws)
+
+        res = {}
+        for name, fn in (("fwd", fwd), ("bwd", bwd)):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            res[name] = e0.elapsed_time(e1) / reps
+        res["fwd+bwd"] = res["fwd"] + res["bwd"]
+        line = {"grid": True, **w}
+        for name, ms in res.items():
+            tf = flops(w, name) / (ms * 1e-3) / 1e12
+            line[name] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                          "frac": round(tf / peaks["bf16_tflops"], 3)}
+        print(json.dumps(line), flush=True)
+        del q, k, v, do, o, lse, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+
+
 # --------------------------------------------------------------- GPU timing
 def main():
     ap = argparse.ArgumentParser()
@@ -282,8 +345,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--grid", action="store_true",
+                    help="time every point of the benchmark-figure grid (1 GPU), one JSON line each")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.grid:
+        run_grid(args)
+        return
     w = WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

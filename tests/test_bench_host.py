@@ -95,3 +95,14 @@ def test_max_over_ranks_gloo_world_size_2():
 
 def test_max_over_ranks_single_process():
     assert bench.max_over_ranks([3, 4.5]) == [3.0, 4.5]
+
+
+def test_grid_points_mirror_the_benchmark_axes():
+    import bench
+
+    pts = bench.grid_points()
+    assert len(pts) == 24  # x 3 passes (fwd, bwd, fwd+bwd) = 72 measurements
+    assert {p["d"] for p in pts} == {64, 128} and {p["causal"] for p in pts} == {False, True}
+    assert sorted({p["N"] for p in pts}) == [512, 1024, 2048, 4096, 8192, 16384]
+    for p in pts:
+        assert p["B"] * p["N"] == 16384 and p["H"] * p["d"] == 2048
