@@ -86,8 +86,9 @@ struct FwdCfg {
   static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 of the largest P entry
   static constexpr int HEAD_GROUP = 16;                    // causal launch order, see below
   // d = 64: one pair of weights in POLY_EVERY is exponentiated on the FMA pipe
-  // (the MUFU unit is the tighter limit there); d = 128: MUFU only (measured faster)
-  static constexpr int POLY_EVERY = (D == 64) ? 3 : 1 << 20;
+  // (the MUFU unit is the tighter limit there; one in 8 measured fastest of
+  // 2, 3, 4, 5, 6, 8, 12 and none); d = 128: MUFU only (measured faster)
+  static constexpr int POLY_EVERY = (D == 64) ? 8 : 1 << 20;
 };
 
 struct FwdParams {
