@@ -164,8 +164,8 @@ FA2_API fa2_status fa2_backward_dq(const void* q, const void* k, const void* v, 
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Backward pass that allocates nothing and takes no workspace. (The paper has
- * no counterpart; this is a deployment convenience of this library.)
+ * Backward pass that allocates nothing and takes no workspace. (The pages
+ * describe no counterpart; this is a deployment convenience of this library.)
  *
  * For callers that cannot allocate device memory when they run the backward:
  * applications that reserve all device memory at start-up and may not call
