@@ -126,25 +126,43 @@ def _bhnd(q):
     return tuple(int(x) for x in q.shape)
 
 
-def _require(t, name, dtype=None):
+def _require(t, name, dtype=None, shape=None):
+    """Checks one tensor argument before its pointer goes to the library: a
+    contiguous CUDA tensor on the current device (where the library launches),
+    of the given dtype and shape. The C ABI sees only pointers and sizes, so a
+    wrong shape or device would otherwise reach the kernels."""
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    import torch
+
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device}; the library launches on the current "
+                         f"device cuda:{cur}")
+
+
+def _require_bf16(shape, *named):
+    import torch
+
+    for t, n in named:
+        _require(t, n, torch.bfloat16, shape)
+
+
+def _require_lse(lse, shape):
+    import torch
+
+    _require(lse, "lse", torch.float32, shape)
 
 
 def fa2_forward(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
     """C ABI fa2_forward on torch tensors: q, k, v, o bf16 [B,H,N,d]; lse fp32 [B,H,N]."""
-    import torch
-
     B, H, N, d = _bhnd(q)
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
-        _require(t, n, torch.bfloat16)
-        if tuple(t.shape) != (B, H, N, d):
-            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
-    _require(lse, "lse", torch.float32)
-    if tuple(lse.shape) != (B, H, N):
-        raise ValueError("lse must be [B, H, N]")
+    _require_bf16((B, H, N, d), (q, "q"), (k, "k"), (v, "v"), (o, "o"))
+    _require_lse(lse, (B, H, N))
     _check("fa2_forward", load_library().fa2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N,
                                           d, int(bool(causal)), float(scale), _stream(stream)))
 
@@ -156,15 +174,10 @@ def fa2_backward_workspace_size(B: int, H: int, N: int, d: int) -> int:
 def fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float, workspace,
                  stream=None) -> None:
     """C ABI fa2_backward on torch tensors; workspace is a uint8 CUDA tensor."""
-    import torch
-
     B, H, N, d = _bhnd(q)
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"),
-                 (dv, "dv")):
-        _require(t, n, torch.bfloat16)
-        if tuple(t.shape) != (B, H, N, d):
-            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
-    _require(lse, "lse", torch.float32)
+    _require_bf16((B, H, N, d), (q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"),
+                  (dq, "dq"), (dk, "dk"), (dv, "dv"))
+    _require_lse(lse, (B, H, N))
     _require(workspace, "workspace")
     nbytes = workspace.numel() * workspace.element_size()
     _check("fa2_backward", load_library().fa2_backward(
@@ -179,6 +192,9 @@ def _nbytes(t) -> int:
 def fa2_backward_preprocess(o, lse, dout, workspace, stream=None) -> None:
     """C ABI fa2_backward_preprocess (first of the three backward stages)."""
     B, H, N, d = _bhnd(o)
+    _require_bf16((B, H, N, d), (o, "o"), (dout, "dout"))
+    _require_lse(lse, (B, H, N))
+    _require(workspace, "workspace")
     _check("fa2_backward_preprocess", load_library().fa2_backward_preprocess(
         _ptr(o), _ptr(lse), _ptr(dout), B, H, N, d, _ptr(workspace), _nbytes(workspace),
         _stream(stream)))
@@ -188,6 +204,9 @@ def fa2_backward_main(q, k, v, dout, dk, dv, causal: bool, scale: float, workspa
                       stream=None) -> None:
     """C ABI fa2_backward_main (dK, dV and the fp32 dQ accumulator)."""
     B, H, N, d = _bhnd(q)
+    _require_bf16((B, H, N, d), (q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (dk, "dk"),
+                  (dv, "dv"))
+    _require(workspace, "workspace")
     _check("fa2_backward_main", load_library().fa2_backward_main(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)),
         float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
@@ -196,6 +215,8 @@ def fa2_backward_main(q, k, v, dout, dk, dv, causal: bool, scale: float, workspa
 def fa2_backward_dq_convert(dq, scale: float, workspace, stream=None) -> None:
     """C ABI fa2_backward_dq_convert (dq = bf16(scale * accumulator))."""
     B, H, N, d = _bhnd(dq)
+    _require_bf16((B, H, N, d), (dq, "dq"))
+    _require(workspace, "workspace")
     _check("fa2_backward_dq_convert", load_library().fa2_backward_dq_convert(
         _ptr(dq), B, H, N, d, float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
@@ -203,15 +224,10 @@ def fa2_backward_dq_convert(dq, scale: float, workspace, stream=None) -> None:
 def fa2_backward_ex(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float, workspace,
                     dq_strategy: int = DQ_AUTO, stream=None) -> None:
     """C ABI fa2_backward_ex: fa2_backward with an explicit dQ strategy."""
-    import torch
-
     B, H, N, d = _bhnd(q)
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"),
-                 (dv, "dv")):
-        _require(t, n, torch.bfloat16)
-        if tuple(t.shape) != (B, H, N, d):
-            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
-    _require(lse, "lse", torch.float32)
+    _require_bf16((B, H, N, d), (q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"),
+                  (dq, "dq"), (dk, "dk"), (dv, "dv"))
+    _require_lse(lse, (B, H, N))
     _require(workspace, "workspace")
     _check("fa2_backward_ex", load_library().fa2_backward_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
@@ -227,6 +243,9 @@ def fa2_backward_main_dkdv(q, k, v, dout, dk, dv, causal: bool, scale: float, wo
                            stream=None) -> None:
     """C ABI fa2_backward_main_dkdv (dK, dV only; FA2_DQ_SEPARATE)."""
     B, H, N, d = _bhnd(q)
+    _require_bf16((B, H, N, d), (q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (dk, "dk"),
+                  (dv, "dv"))
+    _require(workspace, "workspace")
     _check("fa2_backward_main_dkdv", load_library().fa2_backward_main_dkdv(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)),
         float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
@@ -235,6 +254,8 @@ def fa2_backward_main_dkdv(q, k, v, dout, dk, dv, causal: bool, scale: float, wo
 def fa2_backward_dq(q, k, v, dout, dq, causal: bool, scale: float, workspace, stream=None) -> None:
     """C ABI fa2_backward_dq (query-parallel dQ kernel; FA2_DQ_SEPARATE)."""
     B, H, N, d = _bhnd(q)
+    _require_bf16((B, H, N, d), (q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (dq, "dq"))
+    _require(workspace, "workspace")
     _check("fa2_backward_dq", load_library().fa2_backward_dq(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), B, H, N, d, int(bool(causal)),
         float(scale), _ptr(workspace), _nbytes(workspace), _stream(stream)))
@@ -259,17 +280,11 @@ def fa2_forward_qk(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> 
     """C ABI fa2_forward_qk: q, o [B,H,Nq,d], k, v [B,H,Nk,d] bf16; lse fp32 [B,H,Nq].
     Causal masking is aligned to the bottom-right corner (query i sees keys
     j <= i + Nk - Nq)."""
-    import torch
-
     B, H, Nq, d = _bhnd(q)
-    Nk = int(k.shape[2])
-    for t, n, rows in ((q, "q", Nq), (k, "k", Nk), (v, "v", Nk), (o, "o", Nq)):
-        _require(t, n, torch.bfloat16)
-        if tuple(t.shape) != (B, H, rows, d):
-            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, rows, d)}")
-    _require(lse, "lse", torch.float32)
-    if tuple(lse.shape) != (B, H, Nq):
-        raise ValueError("lse must be [B, H, Nq]")
+    Nk = _bhnd(k)[2]
+    _require_bf16((B, H, Nq, d), (q, "q"), (o, "o"))
+    _require_bf16((B, H, Nk, d), (k, "k"), (v, "v"))
+    _require_lse(lse, (B, H, Nq))
     _check("fa2_forward_qk", load_library().fa2_forward_qk(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, int(bool(causal)),
         float(scale), _stream(stream)))
@@ -279,16 +294,11 @@ def fa2_backward_qk(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: floa
                     stream=None) -> None:
     """C ABI fa2_backward_qk (shapes as fa2_forward_qk; dq like q, dk and dv like k;
     workspace of fa2_backward_workspace_size(B, H, Nq, d) bytes)."""
-    import torch
-
     B, H, Nq, d = _bhnd(q)
-    Nk = int(k.shape[2])
-    for t, n, rows in ((q, "q", Nq), (k, "k", Nk), (v, "v", Nk), (o, "o", Nq), (dout, "dout", Nq),
-                       (dq, "dq", Nq), (dk, "dk", Nk), (dv, "dv", Nk)):
-        _require(t, n, torch.bfloat16)
-        if tuple(t.shape) != (B, H, rows, d):
-            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, rows, d)}")
-    _require(lse, "lse", torch.float32)
+    Nk = _bhnd(k)[2]
+    _require_bf16((B, H, Nq, d), (q, "q"), (o, "o"), (dout, "dout"), (dq, "dq"))
+    _require_bf16((B, H, Nk, d), (k, "k"), (v, "v"), (dk, "dk"), (dv, "dv"))
+    _require_lse(lse, (B, H, Nq))
     _require(workspace, "workspace")
     _check("fa2_backward_qk", load_library().fa2_backward_qk(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
@@ -298,38 +308,41 @@ def fa2_backward_qk(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: floa
 
 def attention_forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
     """Allocates o and lse, runs fa2_forward (fa2_forward_qk when k and q differ in
-    length), returns (o, lse)."""
+    length) on q's device, returns (o, lse)."""
     import torch
 
     B, H, N, d = _bhnd(q)
     if scale is None:
         scale = d ** -0.5
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if k.shape[2] != N:
-        fa2_forward_qk(q, k, v, o, lse, causal, scale, stream)
-    else:
-        fa2_forward(q, k, v, o, lse, causal, scale, stream)
+    with torch.cuda.device(q.device):
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+        if k.shape[2] != N:
+            fa2_forward_qk(q, k, v, o, lse, causal, scale, stream)
+        else:
+            fa2_forward(q, k, v, o, lse, causal, scale, stream)
     return o, lse
 
 
 def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
                        stream=None, workspace=None, dq_strategy: int = DQ_AUTO):
-    """Allocates dq, dk, dv (and the workspace unless given), runs fa2_backward_ex."""
+    """Allocates dq, dk, dv (and the workspace unless given), runs fa2_backward_ex
+    (fa2_backward_qk when k and q differ in length) on q's device."""
     import torch
 
     B, H, N, d = _bhnd(q)
     if scale is None:
         scale = d ** -0.5
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    if workspace is None:
-        workspace = torch.empty(fa2_backward_workspace_size(B, H, N, d), dtype=torch.uint8,
-                                device=q.device)
-    if k.shape[2] != N:  # different key length: fa2_backward_qk (dQ by reductions)
-        fa2_backward_qk(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, stream)
-    else:
-        fa2_backward_ex(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, dq_strategy,
-                        stream)
+    with torch.cuda.device(q.device):
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        if workspace is None:
+            workspace = torch.empty(fa2_backward_workspace_size(B, H, N, d), dtype=torch.uint8,
+                                    device=q.device)
+        if k.shape[2] != N:  # different key length: fa2_backward_qk (dQ by reductions)
+            fa2_backward_qk(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace, stream)
+        else:
+            fa2_backward_ex(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, workspace,
+                            dq_strategy, stream)
     return dq, dk, dv
 
 
@@ -347,6 +360,9 @@ def fa2_backward_noalloc(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale:
         fn.argtypes = [vp] * 9 + [i, i, i, i, i, ctypes.c_float, vp]
         fn.restype = i
     B, H, N, d = _bhnd(q)
+    _require_bf16((B, H, N, d), (q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"),
+                  (dq, "dq"), (dk, "dk"), (dv, "dv"))
+    _require_lse(lse, (B, H, N))
     _check("fa2_backward_noalloc", fn(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
         B, H, N, d, int(bool(causal)), float(scale), _stream(stream)))
