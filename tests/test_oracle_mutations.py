@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 from tests import test_oracle as pins
+from tests import test_oracle_library as pins_lib
 from tests import test_oracle_qk as pins_qk
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.cpp")
@@ -61,8 +62,13 @@ def test_pins_pass_on_the_committed_oracle():
     _run_pins()
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name, tmp_path):
+def _run_library_pin():
+    """Only the PyTorch pin of test_oracle_library.py, on two shapes."""
+    pins_lib.check_case(oracle, 1, 2, 9, 9, 8, True)
+    pins_lib.check_case(oracle, 1, 1, 5, 9, 4, True)
+
+
+def _build_mutant(name, tmp_path):
     old, new = MUTANTS[name]
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
@@ -72,7 +78,24 @@ def test_pins_catch_mutant(name, tmp_path):
     lib = tmp_path / "libmutant.so"
     flags = [f for f in oracle.CXXFLAGS if f != "-O3"] + ["-O1"]
     subprocess.run(["g++", *flags, str(path), "-o", str(lib)], check=True)
-    with oracle.use_library(str(lib)):
+    return str(lib)
+
+
+def test_library_pin_passes_on_the_committed_oracle():
+    _run_library_pin()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    with oracle.use_library(_build_mutant(name, tmp_path)):
         with pytest.raises(AssertionError):
             with np.errstate(all="ignore"):
                 _run_pins()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_library_pin_alone_catches_mutant(name, tmp_path):
+    with oracle.use_library(_build_mutant(name, tmp_path)):
+        with pytest.raises(AssertionError):
+            with np.errstate(all="ignore"):
+                _run_library_pin()
