@@ -9,8 +9,9 @@
  *   "FlashAttention-2" summary page, How It Works items 1-2 (work split along
  *   the sequence as well as batch and heads; scaling done once at the end);
  *   "FlashAttention-2: Faster Attention with Better Parallelism and Work
- *   Partitioning" reproduction page, closing paragraph (blocks wholly above the
- *   causal diagonal skipped, one square block per row masked elementwise) and
+ *   Partitioning" reproduction page, closing paragraph (key blocks entirely
+ *   above the diagonal are never computed; only the diagonal block of each
+ *   row of blocks needs the elementwise mask) and
  *   Figures 5-6 (forward and backward attention are the benchmarked passes).
  *
  * For each head (b, h) and rows i, keys j in [0, N):

@@ -7,8 +7,8 @@
 // What it computes is the plain definition of standard attention, because the
 // tiled method reaches that result exactly up to rounding order:
 //   * "FlashAttention (v2)" glossary page, definition paragraph: the method
-//     computes attention "without approximating the result", tile by tile;
-//     results paragraph: its output matches standard attention exactly.
+//     works through attention tile by tile and makes no approximation;
+//     results paragraph: what it returns is standard attention's result.
 //   * "FlashAttention-2" summary page, "How It Works": the work is only
 //     re-partitioned and the scaling moved to the end; the function computed is
 //     unchanged.

@@ -197,7 +197,7 @@ def test_one_dominant_key(oracle_mod):
 
 # ------------------------------------- tiled online softmax (shape N=12, tile 4)
 def online_softmax_tiled(q, k, v, causal, scale, tile):
-    """Exact attention one key tile at a time with a running max and sum, rescaling
+    """Exact attention, key tile by key tile, with a running max and sum, rescaling
     the accumulator when the max grows and dividing by the sum once at the end
     ("FlashAttention-2" summary page, How It Works item 2)."""
     N, d = q.shape
