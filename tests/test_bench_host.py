@@ -1,5 +1,6 @@
 """Host-side pieces of bench.py: FLOP counts, peaks, the ncu traffic record, the
-per-rank seeds and the max-over-ranks timing reduction (world size 2 over gloo)."""
+per-rank seeds, the max-over-ranks timing reduction (world size 2 over gloo), the
+benchmark-figure grid and the reference arm's JSON line."""
 import json
 import os
 import socket
@@ -8,6 +9,8 @@ import pytest
 import torch.multiprocessing as mp
 
 import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_flop_counts():
@@ -106,3 +109,30 @@ def test_grid_points_mirror_the_benchmark_axes():
     assert sorted({p["N"] for p in pts}) == [512, 1024, 2048, 4096, 8192, 16384]
     for p in pts:
         assert p["B"] * p["N"] == 16384 and p["H"] * p["d"] == 2048
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` runs the oracle on the host and prints one JSON
+    line with the contract's keys (no GPU involved)."""
+    import json
+    import subprocess
+    import sys
+
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                         timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in rec, key
+    assert rec["impl"] == "reference" and rec["steps"] == 1 and rec["warmup"] == 3
+    assert rec["metric"] == bench.METRIC and rec["unit"] == "TFLOP/s"
+    assert rec["value"] > 0 and rec["higher_is_better"] is True
+    assert rec["config"]["workload"] == bench.DEFAULT_WORKLOAD
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
+    assert rec["e2e"]["value"] == rec["value"]
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
