@@ -102,3 +102,32 @@ def test_scale_other_than_the_default(oracle_mod):
         g = oracle_mod.attention_backward(t["q"], t["k"], t["v"], t["do"], True, scale)
         for name in ("o", "lse", "dq", "dk", "dv"):
             close(g[name], ref[name], f"{name} at scale {scale}")
+
+
+def test_random_shapes_match_pytorch(oracle_mod):
+    """Seeded random shapes, masks and scales (odd head dims, single rows, more
+    queries than keys without the mask), all entry points against PyTorch."""
+    rng = np.random.default_rng(20260)
+    for trial in range(40):
+        B, H = int(rng.integers(1, 3)), int(rng.integers(1, 3))
+        Nk = int(rng.integers(1, 41))
+        causal = bool(rng.integers(0, 2))
+        Nq = int(rng.integers(1, Nk + 1)) if causal else int(rng.integers(1, 41))
+        d = int(rng.integers(1, 17))
+        scale = float(rng.uniform(0.0, 2.0))
+        t = inputs(5000 + 10 * trial, B, H, Nq, Nk, d)
+        ref = torch_reference(t, causal, scale)
+        where = f"trial {trial}: B={B} H={H} Nq={Nq} Nk={Nk} d={d} causal={causal} scale={scale:.3f}"
+        o, lse = oracle_mod.attention_forward(t["q"], t["k"], t["v"], causal, scale)
+        close(o, ref["o"], f"o, {where}")
+        close(lse, ref["lse"], f"lse, {where}")
+        g = oracle_mod.attention_backward(t["q"], t["k"], t["v"], t["do"], causal, scale)
+        for name in ("dq", "dk", "dv"):
+            close(g[name], ref[name], f"{name}, {where}")
+        qrows = np.unique(rng.integers(0, Nq, size=3))
+        krows = np.unique(rng.integers(0, Nk, size=3))
+        dq_r, dk_r, dv_r = oracle_mod.attention_backward_rows(t["q"], t["k"], t["v"], t["do"],
+                                                              causal, scale, qrows, krows)
+        close(dq_r, ref["dq"][..., qrows, :], f"dq rows, {where}")
+        close(dk_r, ref["dk"][..., krows, :], f"dk rows, {where}")
+        close(dv_r, ref["dv"][..., krows, :], f"dv rows, {where}")
