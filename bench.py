@@ -6,11 +6,14 @@ fa2_forward, then the three backward stages (preprocess, main, dQ convert),
 each launched through the C ABI on the current stream with CUDA events between
 them, so every kernel's duration is measured live inside the timed region.
 
-Default workload (one GPU): B=8, H=16, N=2048, d=128, causal, bf16 i.i.d.
-N(0,1) Q/K/V/dO from the shared seeded generator: the forward+backward
-configuration the attention benchmark of the pages quotes (forward, backward
-and forward+backward TFLOP/s, Figures 4-6 of the FlashAttention-2 paper's
-reproduction page). FLOPs: forward 4*B*H*N^2*d, backward 2.5x, causal halved
+Default workload (one GPU): B=1, H=16, N=16384, d=128, causal, bf16 i.i.d.
+N(0,1) Q/K/V/dO from the shared seeded generator: the longest sequence of the
+attention benchmark the pages quote (forward, backward and forward+backward
+TFLOP/s against sequence length up to 16k, head dimension 64 and 128, with and
+without the causal mask: Figures 4-7 of the FlashAttention-2 paper's
+reproduction page). ``--workload`` selects the shorter forward+backward
+(B=8 H=16 N=2048 d=128 causal) or the forward-only (B=8 H=32 N=2048 d=64)
+workload instead. FLOPs: forward 4*B*H*N^2*d, backward 2.5x, causal halved
 (value) and unhalved (value_unhalved).
 
 Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
@@ -33,6 +36,8 @@ import sys
 import threading
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -42,7 +47,7 @@ WORKLOADS = {
     "fwd_b8_h32_n2048_d64": dict(cfg=1, B=8, H=32, N=2048, d=64, causal=False),
     "fwd_bwd_b1_h16_n16384_d128_causal": dict(cfg=3, B=1, H=16, N=16384, d=128, causal=True),
 }
-DEFAULT_WORKLOAD = "fwd_bwd_b8_h16_n2048_d128_causal"
+DEFAULT_WORKLOAD = "fwd_bwd_b1_h16_n16384_d128_causal"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
     "fa2_fwd_kernel": ["fwd_sm100.cuh", "sm100_ptx.cuh", "exp2_poly.cuh"],
@@ -89,7 +94,7 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 50 ms in the background."""
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms in the background."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -101,7 +106,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50", "-i", str(device_index)],
+                 "-lms", "20", "-i", str(device_index)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             return
@@ -122,25 +127,35 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self, t0: float, t1: float):
-        inside = [p for t, p in self.samples if t0 <= t <= t1]
-        used = inside
-        if not used:  # timed region shorter than one sample period: nearest samples
-            used = [p for t, p in self.samples if t0 - 0.2 <= t <= t1 + 0.2]
-        if not used:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"],
-                    "samples": 0}
+    @staticmethod
+    def _reasons(samples):
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = set()
+        for p in samples:
+            for name, val in zip(names, p[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return reasons
+
+    def summary(self, t0: float, t1: float):
+        """Median SM clock and the throttle reasons seen by the samples taken inside
+        [t0, t1]. With no sample inside, the clock fields are null (a number taken
+        outside the timed region would not describe it); the reasons seen by the
+        samples within 0.2 s of it are still listed, under ``reasons_nearby``."""
+        inside = [p for t, p in self.samples if t0 <= t <= t1]
+        if not inside:
+            near = [p for t, p in self.samples if t0 - 0.2 <= t <= t1 + 0.2]
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "reasons_nearby": sorted(self._reasons(near)) if near else
+                    ["no nvidia-smi samples"]}
+        used = inside
+        reasons = self._reasons(used)
         mhz = []
         for p in used:
             try:
                 mhz.append(float(p[1]))
             except ValueError:
                 pass
-            for name, val in zip(names, p[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
         try:
             smax = float(used[0][2])
         except ValueError:
@@ -185,40 +200,73 @@ def make_inputs(w, rank: int):
 
 
 # ------------------------------------------------------------- oracle timing
+#: heads whose full N x N backward the oracle holds in memory; above this the
+#: oracle runs the whole forward of a head and the gradients of sampled rows
+FULL_BACKWARD_MAX_N = 4096
+#: query rows (dQ) and key rows (dK, dV) per head in the row-sampled backward
+SAMPLED_GRAD_ROWS = 64
+
+
+def _visible(i, N, causal):
+    """Keys that query i sees (self-attention)."""
+    return i + 1 if causal else N
+
+
+def oracle_head(w, host, head: int, threads: int):
+    """Runs the oracle on one (b, h) head of the workload and returns
+    (seconds, FLOPs of the arithmetic it did, description).
+
+    N <= FULL_BACKWARD_MAX_N: the full forward and backward of the head; FLOPs
+    counted like the GPU's (forward 4 N^2 d, backward 2.5x, causal halved).
+    Longer heads: the full forward of the head (every O_i, LSE_i, D_i) and the
+    gradients of SAMPLED_GRAD_ROWS evenly spaced query rows (dQ) and key rows
+    (dK, dV), straight from their definitions. FLOPs counted per visible
+    (query, key) pair: 4 d for a forward row (score and weighted sum), 6 d for a
+    dQ row (score, dP, weighted sum), 8 d for a dK/dV row (score, dP and both
+    weighted sums)."""
+    import oracle
+
+    N, d, causal = w["N"], w["d"], w["causal"]
+    b, h = divmod(head % (w["B"] * w["H"]), w["H"])
+    scale = 1.0 / math.sqrt(d)
+    args = (host["q"][b, h], host["k"][b, h], host["v"][b, h], host["do"][b, h], causal, scale)
+    if N <= FULL_BACKWARD_MAX_N:
+        t0 = time.perf_counter()
+        oracle.attention_backward(*args, nthreads=threads)
+        secs = time.perf_counter() - t0
+        return secs, flops(dict(w, B=1, H=1), "fwd+bwd"), "full forward + backward in fp64"
+    rows = [int(x) for x in np.linspace(0, N - 1, SAMPLED_GRAD_ROWS).round()]
+    t0 = time.perf_counter()
+    oracle.attention_backward_rows(*args, rows, rows, nthreads=threads)
+    secs = time.perf_counter() - t0
+    fl = 4.0 * d * sum(_visible(i, N, causal) for i in range(N))
+    fl += 6.0 * d * sum(_visible(i, N, causal) for i in rows)
+    fl += 8.0 * d * sum((N - j) if causal else N for j in rows)
+    desc = (f"fp64 forward of all {N} rows + dQ of {len(rows)} query rows and dK, dV of "
+            f"{len(rows)} key rows; FLOPs of the arithmetic done")
+    return secs, fl, desc
+
+
 def oracle_sample(w, host, max_seconds: float):
-    """Times the fp64 oracle (fwd + full bwd) on whole heads of this workload,
-    adding heads until about max_seconds of CPU work; returns (TFLOP/s, desc, threads)."""
+    """Times the fp64 oracle on whole heads of this workload (oracle_head), adding
+    heads until about max_seconds of CPU work; returns (TFLOP/s, desc, threads, s)."""
     import oracle
 
     oracle.build()
     threads = oracle.default_threads()
-    scale = 1.0 / math.sqrt(w["d"])
-    per_head = dict(w, B=1, H=1)
-    done, elapsed = 0, 0.0
+    done, elapsed, fl, desc = 0, 0.0, 0.0, ""
     total_heads = w["B"] * w["H"]
     while done < total_heads and elapsed < max_seconds:
-        b, h = divmod(done, w["H"])
-        t0 = time.perf_counter()
-        if w["N"] <= 4096:
-            oracle.attention_backward(host["q"][b, h], host["k"][b, h], host["v"][b, h],
-                                      host["do"][b, h], w["causal"], scale, nthreads=threads)
-        else:  # forward of the whole head plus dQ/dK/dV of 8 rows (the sampled-row path)
-            rows = [0, 1, w["N"] // 2, w["N"] - 1]
-            oracle.attention_backward_rows(host["q"][b, h], host["k"][b, h], host["v"][b, h],
-                                           host["do"][b, h], w["causal"], scale, rows, rows,
-                                           nthreads=threads)
-        elapsed += time.perf_counter() - t0
+        secs, f, desc = oracle_head(w, host, done, threads)
+        elapsed += secs
+        fl += f
         done += 1
-    if w["N"] <= 4096:
-        fl = flops(per_head, "fwd+bwd") * done
-        desc = f"{done} of {total_heads} heads, full fwd+bwd in fp64"
-    else:
-        fl = flops(per_head, "fwd") * done
-        desc = f"{done} of {total_heads} heads, fp64 forward of every row (+4 gradient rows)"
-    return fl / elapsed / 1e12, desc, threads, elapsed
+    return fl / elapsed / 1e12, f"{done} of {total_heads} heads: {desc}", threads, elapsed
 
 
 def run_reference(args, w, rank: int):
+    """The reference arm: the fp64 oracle as it stands on the host cores, one head
+    of the workload per step (oracle_head), rank 0 only."""
     if rank != 0:
         return
     host = make_inputs(w, 0)
@@ -226,30 +274,20 @@ def run_reference(args, w, rank: int):
 
     oracle.build()
     threads = oracle.default_threads()
-    scale = 1.0 / math.sqrt(w["d"])
-    per_head = dict(w, B=1, H=1)
-
-    def step(i):
-        b, h = divmod(i % (w["B"] * w["H"]), w["H"])
-        oracle.attention_backward(host["q"][b, h], host["k"][b, h], host["v"][b, h],
-                                  host["do"][b, h], w["causal"], scale, nthreads=threads)
-
-    if w["N"] > 4096:
-        print(json.dumps({"impl": "reference", "unavailable":
-                          "the fp64 oracle's full backward needs N x N memory per head at this N"}))
-        return
     for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
+        oracle_head(w, host, i, threads)
+    elapsed, fl, desc = 0.0, 0.0, ""
     for i in range(args.steps):
-        step(args.warmup + i)
-    dt = time.perf_counter() - t0
-    value = flops(per_head, "fwd+bwd") * args.steps / dt / 1e12
-    sample = f"one head ({w['N']}x{w['d']}, causal={w['causal']}) of the workload per step, fp64"
+        secs, f, desc = oracle_head(w, host, args.warmup + i, threads)
+        elapsed += secs
+        fl += f
+    value = fl / elapsed / 1e12
+    sample = (f"one ({w['N']}x{w['d']}, causal={w['causal']}) head of the workload per step: "
+              f"{desc}")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(args, w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -274,12 +312,18 @@ def workload_config(args, w):
 # ------------------------------------------------------- benchmark-figure grid
 def grid_points():
     """The pages' attention benchmark axes: hidden size 2048 (H = 2048 / d),
-    d in {64, 128}, N in 512 .. 16k with B = 16384 / N, causal and not."""
+    d in {64, 128}, N in 512 .. 16k with B = 16384 / N, causal and not; then
+    ragged lengths (N = 2000 and 4000 at d = 128, same B and H as 2048 and
+    4096), which show what a length that is not a multiple of the 128-row tile
+    costs."""
     pts = []
     for d in (64, 128):
         for causal in (False, True):
             for N in (512, 1024, 2048, 4096, 8192, 16384):
                 pts.append({"B": 16384 // N, "H": 2048 // d, "N": N, "d": d, "causal": causal})
+    for causal in (False, True):
+        for N, B in ((2000, 8), (4000, 4)):
+            pts.append({"B": B, "H": 16, "N": N, "d": 128, "causal": causal, "ragged": True})
     return pts
 
 
@@ -296,6 +340,9 @@ def run_grid(args):
     peaks, _ = load_peaks()
     reps = max(args.steps // 40, 5)
     for w in grid_points():
+        if args.grid_filter and not any(f"{k}={w.get(k)}" in args.grid_filter.split(",")
+                                        for k in ("d", "N")):
+            continue
         B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
         scale = 1.0 / math.sqrt(d)
         q = torch.randn(B, H, N, d, device="cuda", dtype=torch.bfloat16)
@@ -347,6 +394,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--grid", action="store_true",
                     help="time every point of the benchmark-figure grid (1 GPU), one JSON line each")
+    ap.add_argument("--grid-filter", default="",
+                    help="with --grid: only points matching one of these, e.g. 'd=64,N=2000'")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.grid:

@@ -24,6 +24,12 @@
 
 namespace fa2 {
 
+// Heads per causal scheduling group of the main kernel (their Q, dO and dQ
+// accumulator stay in L2 while the group runs).
+#ifndef FA2_BWD_HEAD_GROUP
+#define FA2_BWD_HEAD_GROUP 16
+#endif
+
 // ------------------------------------------------------------- preprocess (B1)
 struct BwdPreParams {
   const __nv_bfloat16* o;
@@ -198,7 +204,7 @@ struct BwdCfg {
   // d = 128 has no free columns left: dQ reuses the dP^T columns once dS is in smem
   static constexpr bool DQ_IN_DP = (D == 128);
   static constexpr uint32_t COL_DQ = DQ_IN_DP ? COL_DP : 256 + 2 * D;
-  static constexpr int HEAD_GROUP = 16;               // heads per scheduling group
+  static constexpr int HEAD_GROUP = FA2_BWD_HEAD_GROUP;  // heads per scheduling group
 };
 
 struct BwdParams {
@@ -432,11 +438,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
       }
       // never leave the CTA with copies still landing in its shared memory
-      if (last_kv_parity >= 0) mbar_wait(bar_kv_full, last_kv_parity, abort_flag, 0x1102);
+      if (last_kv_parity >= 0) mbar_drain_wait(bar_kv_full, last_kv_parity, 0x1102);
       for (int s = 0; s < C::STAGES; ++s)
-        if (last_st_parity[s] >= 0) mbar_wait(bar_st_full(s), last_st_parity[s], abort_flag, 0x1103);
+        if (last_st_parity[s] >= 0) mbar_drain_wait(bar_st_full(s), last_st_parity[s], 0x1103);
       for (int s = 0; s < C::DO_STAGES; ++s)
-        if (last_do_parity[s] >= 0) mbar_wait(bar_do_full(s), last_do_parity[s], abort_flag, 0x1106);
+        if (last_do_parity[s] >= 0) mbar_drain_wait(bar_do_full(s), last_do_parity[s], 0x1106);
     }
   } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
@@ -570,7 +576,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         gs += n_iter;
       }
       umma_commit(bar_drain);
-      mbar_wait(bar_drain, 0, abort_flag, 0x1207);
+      mbar_drain_wait(bar_drain, 0, 0x1207);
     }
   } else if (warp == C::WARP_RED) {
     // -------------------------------------------- dQ reductions, dK/dV stores
@@ -999,9 +1005,9 @@ __global__ void __launch_bounds__(BwdDqCfg<D>::THREADS, 1)
         }
         last_parity[s] = n & 1;
       }
-      mbar_wait(bar_q, 0, abort_flag, 0x1402);
+      mbar_drain_wait(bar_q, 0, 0x1402);
       for (int s = 0; s < C::STAGES; ++s)
-        if (last_parity[s] >= 0) mbar_wait(bar_kv_full(s), last_parity[s], abort_flag, 0x1403);
+        if (last_parity[s] >= 0) mbar_drain_wait(bar_kv_full(s), last_parity[s], 0x1403);
     }
   } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
@@ -1057,7 +1063,7 @@ __global__ void __launch_bounds__(BwdDqCfg<D>::THREADS, 1)
       }
       umma_commit(bar_dq_done);
       umma_commit(bar_drain);
-      mbar_wait(bar_drain, 0, abort_flag, 0x1505);
+      mbar_drain_wait(bar_drain, 0, 0x1505);
     }
   } else {
     // ------------------------------------------------ elementwise groups (0-15)

@@ -855,6 +855,14 @@ fa2_status fa2_forward_backward_host(const void* q, const void* k, const void* v
 
 }  // extern "C"
 
+#ifdef FA2_TEST_HOOKS
+// Test-hooks builds only: plants (key_tile > 0) or removes (0) the forward
+// producer's skipped load described at g_test_stall_kv. Returns 0 on success.
+extern "C" FA2_API int fa2_debug_set_stall(int key_tile) {
+  return cudaMemcpyToSymbol(fa2::g_test_stall_kv, &key_tile, sizeof(key_tile)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
 #ifdef FA2_TRACE
 // Debug builds only: copies the trace stamps of the last traced launch.
 extern "C" FA2_API int fa2_debug_trace_read(unsigned long long* host, int n) {

@@ -55,6 +55,11 @@
 
 namespace fa2 {
 
+// Heads per causal scheduling group (their K/V tiles stay in L2 while the group runs).
+#ifndef FA2_FWD_HEAD_GROUP
+#define FA2_FWD_HEAD_GROUP 16
+#endif
+
 template <int D>
 struct FwdCfg {
   static_assert(D == 64 || D == 128, "head dim");
@@ -84,7 +89,7 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
   static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 of the largest P entry
-  static constexpr int HEAD_GROUP = 16;                    // causal launch order, see below
+  static constexpr int HEAD_GROUP = FA2_FWD_HEAD_GROUP;    // causal launch order, see below
   // d = 64: one pair of weights in POLY_EVERY is exponentiated on the FMA pipe
   // (the MUFU unit is the tighter limit there; one in 8 measured fastest of
   // 2, 3, 4, 5, 6, 8, 12 and none); d = 128: MUFU only (measured faster)
@@ -251,6 +256,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           const int u = kg / C::STAGES;
           if (u > 0) ok = mbar_wait(bar_kv_empty(s), (u - 1) & 1, abort_flag, 0x101);
           if (!ok) break;
+#ifdef FA2_TEST_HOOKS
+          if (g_test_stall_kv > 0 && kg + 1 == g_test_stall_kv) continue;  // planted stall
+#endif
           const uint32_t kdst = sbase + C::OFF_K + s * 2 * C::TILE_BYTES;
           const uint32_t vdst = sbase + C::OFF_V + s * 2 * C::TILE_BYTES;
           mbar_arrive_expect_tx(bar_kv_full(s), 2 * C::TILE_BYTES);
@@ -262,9 +270,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
       }
       // never leave the CTA with copies still landing in its shared memory
-      if (last_q_parity >= 0) mbar_wait(bar_q_full, last_q_parity, abort_flag, 0x102);
+      if (last_q_parity >= 0) mbar_drain_wait(bar_q_full, last_q_parity, 0x102);
       for (int s = 0; s < C::STAGES; ++s)
-        if (last_parity[s] >= 0) mbar_wait(bar_kv_full(s), last_parity[s], abort_flag, 0x103);
+        if (last_parity[s] >= 0) mbar_drain_wait(bar_kv_full(s), last_parity[s], 0x103);
     }
   } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
@@ -375,7 +383,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       }
       // drain: every UMMA of this CTA has finished before TMEM is released
       umma_commit(bar_drain);
-      mbar_wait(bar_drain, 0, abort_flag, 0x206);
+      mbar_drain_wait(bar_drain, 0, 0x206);
     }
   } else {
     // ---------------------------------------------------------- softmax warps

@@ -18,8 +18,21 @@ __device__ unsigned int g_status;
 constexpr unsigned int kStatusTimeout = 0x80000000u;
 
 // Upper bound on any single wait inside a kernel. A healthy wait is
-// microseconds; the bound only ends kernels whose pipeline logic broke.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+// microseconds; the bound only ends kernels whose pipeline logic broke. The
+// shipped library uses 2 s; the test-hooks build shortens it (FA2_WAIT_LIMIT_NS).
+#ifndef FA2_WAIT_LIMIT_NS
+#define FA2_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr unsigned long long kWaitLimitNs = FA2_WAIT_LIMIT_NS;
+
+#ifdef FA2_TEST_HOOKS
+// Test-hooks build only (never the shipped library): when nonzero, the forward
+// kernel's producer skips the TMA load of the (g_test_stall_kv)-th key tile of
+// every CTA -- it neither issues the copy nor expects its bytes -- so the MMA
+// warp's wait on that stage can only end by running out, which exercises the
+// bounded waits and the abort path on the GPU without any fault.
+__device__ int g_test_stall_kv;
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -96,6 +109,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (*abort) return false;
     if (globaltimer() - t0 > kWaitLimitNs) {
       *abort = 1;
+      report_timeout(site);
+      return false;
+    }
+  }
+}
+
+// The waits of a role's teardown: for its own copies or tensor core operations
+// still in flight before the CTA frees TMEM and exits. Unlike mbar_wait these do
+// not stop at the CTA's abort flag (in flight is in flight, abort or not); they
+// are bounded by the same time limit.
+__device__ __forceinline__ bool mbar_drain_wait(uint32_t bar, uint32_t parity, unsigned int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
       report_timeout(site);
       return false;
     }

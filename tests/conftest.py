@@ -18,3 +18,36 @@ def oracle_mod():
 
     oracle.build()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Prints the parity records of the GPU tests: how many O elements exceeded
+    the plain 1e-2 bar (and were explained by bf16 storage), the worst errors per
+    check, and writes every record to $FA2_PARITY_REPORT (JSON lines) if set."""
+    import json
+
+    from tests import gpu_helpers as gh
+
+    if not gh.REPORT:
+        return
+    o_recs = [r for r in gh.REPORT if r["check"] == "o"]
+    over = [r for r in o_recs if r["n_over_plain_bar"]]
+    tr = terminalreporter
+    tr.write_sep("-", "parity records")
+    tr.write_line(f"{len(gh.REPORT)} checks; O checks: {len(o_recs)}, of which {len(over)} "
+                  f"had elements over the plain 1e-2 bar (all at |O| >= 4, explained by bf16)")
+    for r in over:
+        tr.write_line(f"  O over 1e-2: {r['n_over_plain_bar']} of {r['elements']} elements, "
+                      f"worst {r['max_err']:.4f}, min |O| there {r['min_abs_o_where_over']:.2f}, "
+                      f"excess over rounding {r['max_excess_over_rounding']:.2e} ({r['where']})")
+    for kind, key in (("o", "max_err"), ("lse", "max_err"), ("dq", "rel_fro"), ("dk", "rel_fro"),
+                      ("dv", "rel_fro")):
+        recs = [r for r in gh.REPORT if r["check"] == kind]
+        if recs:
+            w = max(recs, key=lambda r: r[key])
+            tr.write_line(f"  worst {kind} {key}: {w[key]:.3e} ({w['where']})")
+    path = os.environ.get("FA2_PARITY_REPORT")
+    if path:
+        with open(path, "w") as f:
+            for r in gh.REPORT:
+                f.write(json.dumps(r) + "\n")

@@ -23,9 +23,41 @@ def test_flop_counts():
     assert bench.flops(dict(w, causal=False), "fwd") == fwd
 
 
-def test_default_workload_is_forward_backward():
+def test_default_workload_is_the_longest_forward_backward():
+    """The contract line runs the largest single-GPU forward+backward workload:
+    B=1 H=16 N=16384 d=128 causal (the benchmark's longest sequence)."""
     w = bench.WORKLOADS[bench.DEFAULT_WORKLOAD]
-    assert (w["B"], w["H"], w["N"], w["d"], w["causal"]) == (8, 16, 2048, 128, True)
+    assert (w["B"], w["H"], w["N"], w["d"], w["causal"]) == (1, 16, 16384, 128, True)
+
+
+def test_clock_summary_is_null_without_samples_inside():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    row = ["0", "1965", "1965", "300.0", "0x0", "Not Active", "Not Active", "Not Active", "Active"]
+    s.samples = [(10.0, row), (10.5, row)]
+    out = s.summary(10.1, 10.2)  # no sample inside the timed region
+    assert out["sm_mhz"] is None and out["sm_max_mhz"] is None and out["samples"] == 0
+    assert out["reasons_nearby"] == ["sw_power_cap"]
+    out = s.summary(9.9, 10.6)
+    assert out["sm_mhz"] == 1965.0 and out["samples"] == 2 and out["reasons"] == ["sw_power_cap"]
+
+
+def test_row_sampled_oracle_flop_count(monkeypatch):
+    """Heads longer than the full-backward limit: forward of every row (4 d per
+    visible pair) + dQ rows (6 d) + dK, dV rows (8 d), counted exactly."""
+    import numpy as np
+
+    import attn_inputs
+
+    monkeypatch.setattr(bench, "FULL_BACKWARD_MAX_N", 64)
+    monkeypatch.setattr(bench, "SAMPLED_GRAD_ROWS", 4)
+    N, d = 200, 64
+    w = dict(B=1, H=1, N=N, d=d, causal=True)
+    host = attn_inputs.make_qkvdo(9, 1, 1, N, d)
+    secs, fl, desc = bench.oracle_head(w, host, 0, 2)
+    rows = [int(x) for x in np.linspace(0, N - 1, 4).round()]
+    want = 4 * d * N * (N + 1) // 2 + sum(6 * d * (i + 1) for i in rows) + \
+        sum(8 * d * (N - j) for j in rows)
+    assert fl == want and secs > 0 and "dQ of 4 query rows" in desc
 
 
 def test_peaks_fallback(tmp_path, monkeypatch):
@@ -103,12 +135,16 @@ def test_max_over_ranks_single_process():
 def test_grid_points_mirror_the_benchmark_axes():
     import bench
 
-    pts = bench.grid_points()
+    pts = [p for p in bench.grid_points() if not p.get("ragged")]
     assert len(pts) == 24  # x 3 passes (fwd, bwd, fwd+bwd) = 72 measurements
     assert {p["d"] for p in pts} == {64, 128} and {p["causal"] for p in pts} == {False, True}
     assert sorted({p["N"] for p in pts}) == [512, 1024, 2048, 4096, 8192, 16384]
     for p in pts:
         assert p["B"] * p["N"] == 16384 and p["H"] * p["d"] == 2048
+    ragged = [p for p in bench.grid_points() if p.get("ragged")]
+    assert {(p["N"], p["causal"]) for p in ragged} == {(2000, False), (2000, True), (4000, False),
+                                                       (4000, True)}
+    assert all(p["N"] % 128 for p in ragged)
 
 
 def test_reference_arm_prints_one_contract_line():
@@ -148,6 +184,7 @@ def test_reference_arm_under_two_ranks_prints_from_rank_zero_only():
     out = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
                           "--nproc-per-node", "2", "--master-addr", "127.0.0.1", "--master-port",
                           str(port), os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "fwd_bwd_b8_h16_n2048_d128_causal",
                           "--gpus", "2", "--steps", "1", "--warmup", "3"],
                          capture_output=True, text=True, timeout=600, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]

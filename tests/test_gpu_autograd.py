@@ -70,10 +70,10 @@ def test_training_step_gradients(fa2, oracle_mod, causal, d):
     ref_o, _ = oracle_mod.attention_forward(qb, kb, vb, causal, scale)
     ref = oracle_mod.attention_backward(qb, kb, vb, g_bits, causal, scale)
     oo = gh.to_host_f64(o.detach())
-    assert np.all(np.abs(oo - ref_o) <= gh.o_tolerance(ref_o))
+    where = f"autograd B={B} H={H} N={N} d={d} causal={causal}"
+    gh.check_o(oo, ref_o, where)
     for name, t in (("dq", q), ("dk", k), ("dv", v)):
-        err = gh.rel_fro(gh.to_host_f64(t.grad), ref[name])
-        assert err <= gh.GRAD_RTOL, f"{name}: {err:.3e}"
+        gh.check_grad(name, gh.to_host_f64(t.grad), ref[name], where)
     # chain rule through the projections, in fp64 from the oracle's head gradients
     x64 = x.astype(np.float64)
     for n, key in (("q", "dq"), ("k", "dk"), ("v", "dv")):

@@ -33,16 +33,11 @@ def fa2():
 
 def check_against_oracle(oracle_mod, t, got, causal, scale):
     ref = oracle_mod.attention_backward(t["q"], t["k"], t["v"], t["do"], causal, scale)
-    o = gh.to_host_f64(got["o"])
-    err = np.abs(o - ref["o"])
-    assert np.all(err <= gh.o_tolerance(ref["o"])), f"O error {err.max():.3e}"
-    lerr = np.abs(got["lse"].cpu().numpy().astype(np.float64) - ref["lse"]).max()
-    assert lerr <= gh.LSE_ATOL, f"LSE error {lerr:.3e}"
+    where = f"graph replay shape={tuple(t['q'].shape)} causal={causal}"
+    gh.check_o(gh.to_host_f64(got["o"]), ref["o"], where)
+    gh.check_lse(got["lse"].cpu().numpy().astype(np.float64), ref["lse"], where)
     for name in ("dq", "dk", "dv"):
-        g = gh.to_host_f64(got[name])
-        assert np.isfinite(g).all(), f"{name} not finite"
-        e = gh.rel_fro(g, ref[name])
-        assert e <= gh.GRAD_RTOL, f"{name} relative Frobenius error {e:.3e}"
+        gh.check_grad(name, gh.to_host_f64(got[name]), ref[name], where)
 
 
 @pytest.mark.parametrize("d,causal", [(64, False), (128, True)])

@@ -70,13 +70,12 @@ def test_host_path_matches_device_path_and_oracle(fa2, oracle_mod, cfg, B, H, N,
 
     # oracle
     ref_o, ref_lse = oracle_mod.attention_forward(t["q"], t["k"], t["v"], causal, scale)
-    oo = gh.to_host_f64(o)
-    assert np.all(np.abs(oo - ref_o) <= gh.o_tolerance(ref_o))
-    assert np.max(np.abs(lse.numpy().astype(np.float64) - ref_lse)) <= gh.LSE_ATOL
+    where = f"host-buffer entry shape={tuple(t['q'].shape)} causal={causal}"
+    gh.check_o(gh.to_host_f64(o), ref_o, where)
+    gh.check_lse(lse.numpy().astype(np.float64), ref_lse, where)
     ref = oracle_mod.attention_backward(t["q"], t["k"], t["v"], t["do"], causal, scale)
     for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
-        err = gh.rel_fro(gh.to_host_f64(got), ref[name])
-        assert err <= gh.GRAD_RTOL, f"{name} relative Frobenius error {err:.3e}"
+        gh.check_grad(name, gh.to_host_f64(got), ref[name], where)
 
 
 def test_host_path_orders_with_the_callers_stream(fa2):

@@ -59,14 +59,11 @@ def test_qk_forward_backward(fa2, oracle_mod, cfg, B, H, Nq, Nk, d, causal):
     assert st == 0, f"device status {fa2.fa2_status_string(st)} at site {site:#x}"
     assert dq.shape == q.shape and dk.shape == k.shape and dv.shape == v.shape
     ref = oracle_mod.attention_backward(t["q"], t["k"], t["v"], t["do"], causal, scale)
-    oo = gh.to_host_f64(o)
-    assert np.all(np.abs(oo - ref["o"]) <= gh.o_tolerance(ref["o"]))
-    assert np.max(np.abs(gh.to_host_f64(lse) - ref["lse"])) <= gh.LSE_ATOL
+    where = f"Nq={Nq} Nk={Nk} B={B} H={H} d={d} causal={causal}"
+    gh.check_o(gh.to_host_f64(o), ref["o"], where)
+    gh.check_lse(gh.to_host_f64(lse), ref["lse"], where)
     for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
-        g = gh.to_host_f64(got)
-        assert np.isfinite(g).all()
-        err = gh.rel_fro(g, ref[name])
-        assert err <= gh.GRAD_RTOL, f"{name} relative Frobenius error {err:.3e}"
+        gh.check_grad(name, gh.to_host_f64(got), ref[name], where)
 
 
 @pytest.mark.parametrize("causal", [False, True])

@@ -3,9 +3,9 @@
 It exists for callers that cannot allocate device memory when they run the
 backward pass (memory reserved up front, hosts that forbid allocation on the
 hot path, C callers without an allocator). These tests call it through the C
-ABI and compare it with fa2_backward (caller-provided workspace) on two calls
-in a row, so that a second call sees the first call's leftovers in the shared
-scratch array. This file is collected last on purpose.
+ABI and compare it with fa2_backward (caller-provided workspace) and with the
+fp64 oracle on two calls in a row, so that a second call sees the first call's
+leftovers in the shared scratch array. This file is collected last on purpose.
 """
 import ctypes
 import math
@@ -41,7 +41,7 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("B,H,N,d,causal", [(2, 3, 384, 128, True), (1, 4, 1000, 64, False)])
-def test_noalloc_matches_workspace_backward(B, H, N, d, causal):
+def test_noalloc_matches_workspace_backward(oracle_mod, B, H, N, d, causal):
     import torch
 
     if not torch.cuda.is_available():
@@ -54,6 +54,7 @@ def test_noalloc_matches_workspace_backward(B, H, N, d, causal):
     q, k, v, do = (gh.to_device(t[n]) for n in ("q", "k", "v", "do"))
     o, lse = fa2.attention_forward(q, k, v, causal=causal, scale=scale)
     ref = fa2.attention_backward(q, k, v, o, lse, do, causal=causal, scale=scale)
+    oracle_ref = oracle_mod.attention_backward(t["q"], t["k"], t["v"], t["do"], causal, scale)
     stream = torch.cuda.current_stream().cuda_stream
     for call in range(2):
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -66,5 +67,8 @@ def test_noalloc_matches_workspace_backward(B, H, N, d, causal):
         for got, want, name in zip((dq, dk, dv), ref, ("dq", "dk", "dv")):
             err = gh.rel_fro(gh.to_host_f64(got), gh.to_host_f64(want))
             assert err <= gh.GRAD_RTOL, f"call {call}: {name} differs by {err:.3e}"
+            # and against the fp64 oracle, with the tolerance of the parity tests
+            gh.check_grad(name, gh.to_host_f64(got), oracle_ref[name],
+                          f"no-alloc backward call {call} B={B} H={H} N={N} d={d} causal={causal}")
     st, site = fa2.fa2_get_device_status()
     assert st == 0, f"device status {st} at {site:#x}"
