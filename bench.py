@@ -390,6 +390,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer measurement (profiling runs: fewer launches)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--grid", action="store_true",
@@ -496,27 +498,29 @@ def main():
 
     # e2e through the C ABI's host-buffer entry: pinned host inputs in, every
     # output back to pinned host memory, copies pipelined with the kernels
-    outs_host = [torch.empty_like(x, device="cpu").pin_memory() for x in (o, lse, dq, dk, dv)]
-    host_ws = torch.empty(fa2.fa2_forward_backward_host_workspace_size(B, H, N, d, 0),
-                          dtype=torch.uint8, device=dev)
+    e2e_ms = None
+    if not args.no_e2e:
+        outs_host = [torch.empty_like(x, device="cpu").pin_memory() for x in (o, lse, dq, dk, dv)]
+        host_ws = torch.empty(fa2.fa2_forward_backward_host_workspace_size(B, H, N, d, 0),
+                              dtype=torch.uint8, device=dev)
 
-    def e2e_step():
-        fa2.fa2_forward_backward_host(hq, hk, hv, hdo, *outs_host, causal, scale, host_ws, 0,
-                                      stream)
+        def e2e_step():
+            fa2.fa2_forward_backward_host(hq, hk, hv, hdo, *outs_host, causal, scale, host_ws, 0,
+                                          stream)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dist, dev)[0]
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
-    d2h = sum(x.numel() * x.element_size() for x in outs_host)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dist, dev)[0]
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
+        d2h = sum(x.numel() * x.element_size() for x in outs_host)
 
     clocks = sampler.summary(t_wall0, t_wall1)
 
@@ -575,11 +579,12 @@ def main():
         "roofline": roofline,
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
-        "e2e": {"value": fl_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "path": "pinned host Q,K,V,dO -> fa2_forward_backward_host (C ABI; chunks of "
-                        "B*H/8 heads, copies in both directions overlapped with the kernels) -> "
-                        "O, LSE, dQ, dK, dV in pinned host memory"},
+        "e2e": None if e2e_ms is None else {
+            "value": fl_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+            "path": "pinned host Q,K,V,dO -> fa2_forward_backward_host (C ABI; chunks of "
+                    "B*H/8 heads, copies in both directions overlapped with the kernels) -> "
+                    "O, LSE, dQ, dK, dV in pinned host memory"},
         "peaks": {"kind": peaks_kind, **peaks},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -63,6 +63,12 @@ typedef enum {
 
 /*
  * Forward pass: o = softmax(scale * q k^T [causal]) v and lse (natural log).
+ * Defined by the "FlashAttention (v2)" glossary page, definition paragraph
+ * (attention computed tile by tile in on-chip memory, the score matrix never
+ * written to HBM, no approximation) and the "FlashAttention-2" summary page,
+ * How It Works items 1-2 (query blocks spread over the GPU as well as batch
+ * and heads; the softmax normalisation applied once at the end); causal block
+ * skipping from the reproduction page's closing paragraph.
  * q, k, v: inputs [B,H,N,d] bf16. o: output [B,H,N,d] bf16. lse: output
  * [B,H,N] fp32, kept for the backward pass. causal: 0 or 1 (j <= i allowed).
  * Work: pairs of 128-row query blocks x batch*head, taken from a work counter by
@@ -78,6 +84,8 @@ FA2_API fa2_status fa2_forward(const void* q, const void* k, const void* v, void
                        int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * (No counterpart on the pages, which describe no interface: the backward's
+ * scratch memory is caller-owned so that the library never allocates.)
  * Bytes of device workspace fa2_backward needs for these sizes: an fp32 dQ
  * accumulator [B,H,Np,d], two fp32 row vectors [B,H,Np] (D = rowsum(dO o O)
  * and the log2-scaled LSE), with Np = N rounded up to 128, and 16 bytes for the
@@ -86,7 +94,14 @@ FA2_API fa2_status fa2_forward(const void* q, const void* k, const void* v, void
 FA2_API size_t fa2_backward_workspace_size(int B, int H, int N, int d);
 
 /*
- * Backward pass. Inputs q, k, v, o (the forward output), lse (the forward
+ * Backward pass: the gradients of the forward pass with respect to q, k and v,
+ * recomputing the probabilities from the saved LSE rather than storing them.
+ * The pages benchmark this pass ("FlashAttention-2: Faster Attention with
+ * Better Parallelism and Work Partitioning" reproduction page, Figure 6a-d
+ * captions: backward speed against sequence length, head dimension 64 and 128,
+ * with and without the causal mask) but print no equations; the chain-rule
+ * gradients above are this library's reading.
+ * Inputs q, k, v, o (the forward output), lse (the forward
  * LSE), dO (gradient of the loss w.r.t. o). Outputs dq, dk, dv [B,H,N,d] bf16.
  * o and lse must come from fa2_forward on the same q, k, v, causal and scale;
  * they are trusted as given. workspace: caller-owned device memory of at least
