@@ -30,7 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa2_b200
 DQ_AUTO, DQ_REDUCE, DQ_SEPARATE = 0, 1, 2
 
 STATUS = {0: "FA2_OK", 1: "FA2_ERR_INVALID_ARG", 2: "FA2_ERR_UNSUPPORTED",
-          3: "FA2_ERR_MISALIGNED", 4: "FA2_ERR_CUDA", 5: "FA2_ERR_TIMEOUT"}
+          3: "FA2_ERR_MISALIGNED", 4: "FA2_ERR_CUDA", 5: "FA2_ERR_TIMEOUT", 6: "FA2_ERR_CONFLICT"}
 
 
 class FA2Error(RuntimeError):

@@ -224,6 +224,17 @@ struct BwdParams {
   float scale_log2;
 };
 
+// One float from shared memory. Used for the per-column LSE and D values, whose
+// address is the same in every lane of a warp: as 32-bit loads those broadcasts
+// cost one wavefront each, while the 128-bit vector loads the compiler would
+// otherwise merge them into measured ~6.5 wavefronts each (ncu) -- shared
+// memory bandwidth the tensor core's operand reads compete for.
+__device__ __forceinline__ float lds_f32(const float* ptr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(ptr))));
+  return v;
+}
+
 __device__ __forceinline__ void red_add(float* addr, float a) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
@@ -733,7 +744,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           const bool diag = p.causal && off < C::BN - 1;
 #pragma unroll
           for (int e = 0; e < CW; e += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(lse2 + e);
+            const float4 l4 = make_float4(lds_f32(lse2 + e), lds_f32(lse2 + e + 1), lds_f32(lse2 + e + 2),
+                                          lds_f32(lse2 + e + 3));
             float x0, x1, x2, x3;
             f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
             f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
@@ -770,7 +782,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           tmem_ld32(lane_base + C::COL_DP + CW * g, dp);
 #pragma unroll
           for (int e = 0; e < CW; e += 4) {
-            const float4 d4 = *reinterpret_cast<const float4*>(dlt + e);
+            const float4 d4 = make_float4(lds_f32(dlt + e), lds_f32(dlt + e + 1), lds_f32(dlt + e + 2),
+                                          lds_f32(dlt + e + 3));
             const unsigned long long pa = f2(__uint_as_float(pk[e / 2] << 16), __uint_as_float(pk[e / 2] & 0xFFFF0000u));
             const unsigned long long pb = f2(__uint_as_float(pk[e / 2 + 1] << 16), __uint_as_float(pk[e / 2 + 1] & 0xFFFF0000u));
             const unsigned long long da = f2_add(f2(dp[e], dp[e + 1]), f2(-d4.x, -d4.y));

@@ -8,6 +8,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -29,17 +30,70 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Driver entry points, resolved through the runtime (the library does not link
+// libcuda directly, so it loads on machines without a GPU).
+void* driver_entry(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return p;
+}
+
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
+  std::call_once(once, [] { fn = reinterpret_cast<EncodeTiledFn>(driver_entry("cuTensorMapEncodeTiled")); });
   return fn;
+}
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*MemsetD32AsyncFn)(CUdeviceptr, unsigned int, size_t, CUstream);
+
+// The context current on this thread (nullptr if none or unknown).
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] { fn = reinterpret_cast<CtxGetCurrentFn>(driver_entry("cuCtxGetCurrent")); });
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
+MemsetD32AsyncFn memset_d32_fn() {
+  static MemsetD32AsyncFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] { fn = reinterpret_cast<MemsetD32AsyncFn>(driver_entry("cuMemsetD32Async")); });
+  return fn;
+}
+
+// Device address of a __device__ symbol, cached per device together with the
+// context it was looked up in, and looked up again when the current context
+// differs (a cudaDeviceReset or a new primary context frees the old address).
+// The caller holds the cache's mutex and has made `dev` current.
+struct SymbolCache {
+  CUcontext ctx[kMaxDevices] = {};
+  void* addr[kMaxDevices] = {};
+};
+
+template <class T>
+void* symbol_address(SymbolCache& cache, int dev, const T& symbol, fa2_status* st) {
+  const CUcontext ctx = current_context();
+  if (!cache.addr[dev] || cache.ctx[dev] != ctx) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      *st = FA2_ERR_CUDA;
+      return nullptr;
+    }
+    cache.addr[dev] = p;
+    cache.ctx[dev] = ctx;
+  }
+  *st = FA2_OK;
+  return cache.addr[dev];
 }
 
 // Tensor map over a contiguous bf16 [BH, N, d] array seen as 3-D (d, N, BH),
@@ -83,18 +137,18 @@ fa2_status check_device(int* dev_out) {
     cudaGetLastError();
     return FA2_ERR_CUDA;
   }
-  static int cc[kMaxDevices] = {0};
+  static std::atomic<int> cc[kMaxDevices] = {};
   if (dev < 0 || dev >= kMaxDevices) return FA2_ERR_UNSUPPORTED;
-  if (cc[dev] == 0) {
+  if (cc[dev].load(std::memory_order_relaxed) == 0) {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
       cudaGetLastError();
       return FA2_ERR_CUDA;
     }
-    cc[dev] = major * 10 + minor;
+    cc[dev].store(major * 10 + minor, std::memory_order_relaxed);
   }
-  if (cc[dev] != 100) return FA2_ERR_UNSUPPORTED;
+  if (cc[dev].load(std::memory_order_relaxed) != 100) return FA2_ERR_UNSUPPORTED;
   *dev_out = dev;
   return FA2_OK;
 }
@@ -128,36 +182,57 @@ fa2_status ensure_smem(KernelT kernel, int bytes, int dev, bool* done) {
 
 int sm_count(int dev);
 
-// Work-item counters of the persistent forward kernel: a ring of them per
-// device, one per launch, zeroed on the launch's stream right before it. Launches
-// that overlap on the GPU (different streams) use different counters as long as
-// fewer than kFwdCounters of them are in flight at once.
+// Work-item counters of the persistent forward kernel. Each launch takes the
+// next slot of a ring (one per device) and a fresh nonzero 32-bit tag, and one
+// 32-bit memset on the launch's stream writes the tag into both halves of the
+// slot right before the kernel (the kernel counts items in the low half from
+// the tag up and checks the high half on every item). Launches enqueued under
+// stream capture take their slots from a second ring, so eager launches never
+// reuse the slot that a captured graph replays with. When more than
+// kFwdCounters launches of one ring are in flight at once, a launch can find its
+// slot reset by a later one: it then stops taking items and records
+// FA2_ERR_CONFLICT in the device status word instead of silently sharing items.
 constexpr unsigned int kFwdCounters = 256;
-__device__ unsigned int g_fwd_counters[kFwdCounters];
+__device__ unsigned long long g_fwd_counters[2 * kFwdCounters];
 
-unsigned int* fwd_counter(int dev, cudaStream_t stream, fa2_status* st) {
-  static unsigned int* base[kMaxDevices] = {nullptr};
-  static unsigned int next[kMaxDevices] = {0};
+#ifdef FA2_TEST_HOOKS
+std::atomic<int> g_tag_skew{0};  // added to the tag the kernel is given (test builds only)
+#endif
+
+unsigned long long* fwd_counter(int dev, cudaStream_t stream, unsigned int* tag, fa2_status* st) {
+  static SymbolCache base;
+  static unsigned int next[kMaxDevices] = {0}, next_captured[kMaxDevices] = {0}, next_tag[kMaxDevices] = {0};
   static std::mutex mu;
-  unsigned int* c = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (!base[dev]) {
-      void* ptr = nullptr;
-      if (cudaGetSymbolAddress(&ptr, g_fwd_counters) != cudaSuccess || ptr == nullptr) {
-        cudaGetLastError();
-        *st = FA2_ERR_CUDA;
-        return nullptr;
-      }
-      base[dev] = static_cast<unsigned int*>(ptr);
-    }
-    c = base[dev] + (next[dev]++ % kFwdCounters);
-  }
-  if (cudaMemsetAsync(c, 0, sizeof(unsigned int), stream) != cudaSuccess) {
-    cudaGetLastError();
+  MemsetD32AsyncFn memset_d32 = memset_d32_fn();
+  if (!memset_d32) {
     *st = FA2_ERR_CUDA;
     return nullptr;
   }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    cs = cudaStreamCaptureStatusNone;
+  }
+  unsigned long long* c = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    void* b = symbol_address(base, dev, g_fwd_counters, st);
+    if (!b) return nullptr;
+    const unsigned int idx = cs == cudaStreamCaptureStatusActive
+                                 ? kFwdCounters + (next_captured[dev]++ % kFwdCounters)
+                                 : next[dev]++ % kFwdCounters;
+    c = static_cast<unsigned long long*>(b) + idx;
+    if (++next_tag[dev] == 0) ++next_tag[dev];
+    *tag = next_tag[dev];
+  }
+  if (memset_d32(reinterpret_cast<CUdeviceptr>(c), *tag, 2, reinterpret_cast<CUstream>(stream)) !=
+      CUDA_SUCCESS) {
+    *st = FA2_ERR_CUDA;
+    return nullptr;
+  }
+#ifdef FA2_TEST_HOOKS
+  *tag += static_cast<unsigned int>(g_tag_skew.load());
+#endif
   *st = FA2_OK;
   return c;
 }
@@ -191,7 +266,7 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.BH = BH;
   fa2_status st = FA2_OK;
-  p.counter = fwd_counter(dev, stream, &st);
+  p.counter = fwd_counter(dev, stream, &p.tag, &st);
   if (st != FA2_OK) return st;
   // persistent: one CTA per SM (its shared memory and TMEM allow no second one)
   const long long items = static_cast<long long>(BH) * p.n_pairs;
@@ -220,16 +295,16 @@ WsLayout ws_layout(void* workspace, int BH, int N, int d) {
 }
 
 int sm_count(int dev) {
-  static int count[kMaxDevices] = {0};
-  if (count[dev] == 0) {
-    int c = 0;
+  static std::atomic<int> count[kMaxDevices] = {};
+  int c = count[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
     if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c < 1) {
       cudaGetLastError();
       c = 148;
     }
-    count[dev] = c;
+    count[dev].store(c, std::memory_order_relaxed);
   }
-  return count[dev];
+  return c;
 }
 
 // Grid (blocks per head, heads) of the streaming kernels: about 16 blocks per SM
@@ -381,6 +456,7 @@ const char* fa2_status_string(int status) {
     case FA2_ERR_MISALIGNED: return "FA2_ERR_MISALIGNED";
     case FA2_ERR_CUDA: return "FA2_ERR_CUDA";
     case FA2_ERR_TIMEOUT: return "FA2_ERR_TIMEOUT";
+    case FA2_ERR_CONFLICT: return "FA2_ERR_CONFLICT";
     default: return "FA2_ERR_UNKNOWN";
   }
 }
@@ -609,7 +685,9 @@ fa2_status fa2_get_device_status(void* stream, int* info) {
     return FA2_ERR_CUDA;
   }
   if (info) *info = static_cast<int>(word & 0xFFFFu);
-  return (word & fa2::kStatusTimeout) ? FA2_ERR_TIMEOUT : FA2_OK;
+  if (word & fa2::kStatusTimeout) return FA2_ERR_TIMEOUT;
+  if (word & fa2::kStatusConflict) return FA2_ERR_CONFLICT;
+  return FA2_OK;
 }
 
 fa2_status fa2_clear_device_status(void) {
@@ -641,22 +719,13 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[FA2_NOALLOC_SCR
 
 // Device address of g_noalloc_scratch on device `dev` (which must be current).
 // In host code the array's name only stands in for the symbol; the address a
-// kernel may use comes from cudaGetSymbolAddress, looked up once per device.
+// kernel may use comes from cudaGetSymbolAddress, looked up once per device and
+// context (again after a cudaDeviceReset).
 void* noalloc_scratch(int dev, fa2_status* st) {
-  static void* addr[kMaxDevices] = {nullptr};
+  static SymbolCache cache;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      *st = FA2_ERR_CUDA;
-      return nullptr;
-    }
-    addr[dev] = p;
-  }
-  *st = FA2_OK;
-  return addr[dev];
+  return symbol_address(cache, dev, g_noalloc_scratch, st);
 }
 
 }  // namespace
@@ -856,6 +925,14 @@ fa2_status fa2_forward_backward_host(const void* q, const void* k, const void* v
 }  // extern "C"
 
 #ifdef FA2_TEST_HOOKS
+// Test-hooks builds only: the forward kernels launched after this call are given
+// their slot's tag plus `skew`, so that a nonzero skew makes every launch see a
+// foreign tag in its work counter (the FA2_ERR_CONFLICT path). Returns 0.
+extern "C" FA2_API int fa2_debug_forward_tag_skew(int skew) {
+  g_tag_skew.store(skew);
+  return 0;
+}
+
 // Test-hooks builds only: plants (key_tile > 0) or removes (0) the forward
 // producer's skipped load described at g_test_stall_kv. Returns 0 on success.
 extern "C" FA2_API int fa2_debug_set_stall(int key_tile) {

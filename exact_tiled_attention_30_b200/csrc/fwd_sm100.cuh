@@ -99,7 +99,11 @@ struct FwdCfg {
 struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
-  unsigned int* counter;  // next work item, zero at launch
+  // work counter of this launch: both 32-bit halves hold `tag` at launch; the
+  // high half keeps it (a different value means another launch has reset the
+  // slot), the low half minus tag counts the items taken
+  unsigned long long* counter;
+  unsigned int tag;
   int Nq;        // query rows (O, LSE)
   int Nk;        // key rows
   int kq_offset; // Nk - Nq: causal query i sees keys j <= i + kq_offset
@@ -230,8 +234,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       bool ok = true;
       int kg = 0;  // key tiles loaded so far
       for (int n = 0; ok; ++n) {
-        int item = static_cast<int>(atomicAdd(p.counter, 1u));
-        if (item >= n_items) item = -1;
+        const unsigned long long v = atomicAdd(p.counter, 1ull);
+        int item = -1;
+        if (static_cast<unsigned int>(v >> 32) != p.tag) {
+          report_conflict(0x10A);  // the slot now belongs to another launch: stop
+        } else {
+          const unsigned int taken = static_cast<unsigned int>(v) - p.tag;
+          if (taken < static_cast<unsigned int>(n_items)) item = static_cast<int>(taken);
+        }
         if (n >= 2) ok = mbar_wait(bar_item_empty(n & 1), ((n >> 1) - 1) & 1, abort_flag, 0x104);
         if (!ok) break;
         item_slot[n & 1] = item;

@@ -11,11 +11,14 @@
 namespace fa2 {
 
 // ----------------------------------------------------------------- status word
-// One word per device, set by the first kernel that gives up on a wait.
-// Layout: low 16 bits = site code, bit 31 = timeout flag.
+// One word per device, set by the first kernel that records an error.
+// Layout: low 16 bits = site code, bit 31 = timeout flag (a bounded wait ran
+// out), bit 30 = conflict flag (a forward launch found its work counter taken
+// over by another launch).
 __device__ unsigned int g_status;
 
 constexpr unsigned int kStatusTimeout = 0x80000000u;
+constexpr unsigned int kStatusConflict = 0x40000000u;
 
 // Upper bound on any single wait inside a kernel. A healthy wait is
 // microseconds; the bound only ends kernels whose pipeline logic broke. The
@@ -46,6 +49,10 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 
 __device__ __forceinline__ void report_timeout(unsigned int site) {
   atomicCAS(&g_status, 0u, kStatusTimeout | (site & 0xFFFFu));
+}
+
+__device__ __forceinline__ void report_conflict(unsigned int site) {
+  atomicCAS(&g_status, 0u, kStatusConflict | (site & 0xFFFFu));
 }
 
 // -------------------------------------------------------------------- tracing

@@ -58,7 +58,8 @@ typedef enum {
   FA2_ERR_UNSUPPORTED = 2, /* d not in {64, 128}, B*H > 65535, or no sm_100 device */
   FA2_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
   FA2_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor map) */
-  FA2_ERR_TIMEOUT = 5      /* a kernel gave up on a bounded wait (see fa2_get_device_status) */
+  FA2_ERR_TIMEOUT = 5,     /* a kernel gave up on a bounded wait (see fa2_get_device_status) */
+  FA2_ERR_CONFLICT = 6     /* a forward found its work counter reset by a later launch (ditto) */
 } fa2_status;
 
 /*
@@ -72,13 +73,19 @@ typedef enum {
  * q, k, v: inputs [B,H,N,d] bf16. o: output [B,H,N,d] bf16. lse: output
  * [B,H,N] fp32, kept for the backward pass. causal: 0 or 1 (j <= i allowed).
  * Work: pairs of 128-row query blocks x batch*head, taken from a work counter by
- * a persistent grid of one CTA per SM. Enqueues on `stream` a 4-byte
- * cudaMemsetAsync of that counter (one of 256 counters inside the library, used
- * in turn) and one kernel launch. Launches that may overlap on the GPU (other
- * streams) stay independent as long as fewer than 256 are in flight at once;
- * launches ordered on one stream always are. The first call on a device looks
- * up the counters' device address (cudaGetSymbolAddress): make it outside
- * stream capture.
+ * a persistent grid of one CTA per SM. Enqueues on `stream` an 8-byte memset of
+ * that counter (cuMemsetD32Async: the launch's tag in both halves; one of 256
+ * counters inside the library, used in turn) and one kernel launch. Launches
+ * ordered on one stream are always independent. Launches that may overlap on
+ * the GPU (other streams) are independent as long as fewer than 256 are in
+ * flight at once; beyond that a launch can find its counter reset by a later
+ * one: it then stops early and fa2_get_device_status reports FA2_ERR_CONFLICT
+ * (its o and lse, and the later launch's, are then not to be trusted). A forward
+ * enqueued under stream capture takes its counter from a second ring of 256
+ * that eager calls never use, and keeps it for every replay of the graph:
+ * replays of one graph must not overlap one another on the GPU. The first call
+ * on a device (and the first after a cudaDeviceReset) looks up the counters'
+ * device address (cudaGetSymbolAddress): make it outside stream capture.
  */
 FA2_API fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse,
                        int B, int H, int N, int d, int causal, float scale, void* stream);
@@ -276,9 +283,11 @@ FA2_API const char* fa2_status_string(int status);
 
 /*
  * Synchronises `stream` and reports whether any kernel of this library on the
- * current device gave up on a bounded wait since the last clear. Returns
- * FA2_OK, FA2_ERR_TIMEOUT (then *info, if non-NULL, holds a site code), or
- * FA2_ERR_CUDA if the synchronisation itself failed.
+ * current device recorded an error since the last clear: FA2_ERR_TIMEOUT (a
+ * bounded wait ran out) or FA2_ERR_CONFLICT (a forward's work counter was reset
+ * by a later launch while it ran; see fa2_forward); then *info, if non-NULL,
+ * holds a site code. Returns FA2_OK if none, FA2_ERR_CUDA if the
+ * synchronisation itself failed.
  */
 FA2_API fa2_status fa2_get_device_status(void* stream, int* info);
 

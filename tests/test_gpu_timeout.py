@@ -46,6 +46,8 @@ def test_shipped_library_has_no_test_hooks():
 
     lib = fa2.load_library()
     assert not hasattr(lib, "fa2_debug_set_stall")
+    assert not hasattr(lib, "fa2_debug_forward_tag_skew")
+    assert fa2.fa2_status_string(6) == "FA2_ERR_CONFLICT"
 
 
 @pytest.mark.gpu
@@ -88,5 +90,56 @@ def test_stalled_wait_times_out_then_context_recovers(oracle_mod, d, causal):
     assert st == 0, f"status {st} after clearing, site {info.value:#x}"
     ro, rl = oracle_mod.attention_forward(t["q"], t["k"], t["v"], causal, scale)
     where = f"after a timed-out call, B={B} H={H} N={N} d={d} causal={causal}"
+    gh.check_o(gh.to_host_f64(o2), ro, where)
+    gh.check_lse(lse2.cpu().numpy().astype(np.float64), rl, where)
+
+
+FA2_ERR_CONFLICT = 6
+
+
+@pytest.mark.gpu
+def test_foreign_counter_tag_is_reported_as_conflict(oracle_mod):
+    """A forward whose work counter holds another launch's tag (what happens when
+    more than 256 forwards on different streams are in flight at once and the
+    counter ring wraps onto a running launch) stops taking work and reports
+    FA2_ERR_CONFLICT instead of sharing items silently. The test-hooks build
+    makes every launch see a foreign tag (fa2_debug_forward_tag_skew); with the
+    skew removed and the status cleared, the same context computes correctly."""
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    lib = _test_hooks_lib()
+    lib.fa2_debug_forward_tag_skew.argtypes = [ctypes.c_int]
+    lib.fa2_debug_forward_tag_skew.restype = ctypes.c_int
+    B, H, N, d, causal = 2, 2, 640, 128, True
+    scale = 1.0 / math.sqrt(d)
+    t = gh.inputs(33, B, H, N, d)
+    q, k, v = (gh.to_device(t[n]) for n in ("q", "k", "v"))
+    sp = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    info = ctypes.c_int(0)
+
+    def forward(o, lse):
+        return lib.fa2_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                               lse.data_ptr(), B, H, N, d, int(causal), ctypes.c_float(scale), sp)
+
+    assert lib.fa2_clear_device_status() == 0
+    o, lse = torch.empty_like(q), torch.empty(B, H, N, device="cuda", dtype=torch.float32)
+    assert lib.fa2_debug_forward_tag_skew(1) == 0
+    try:
+        assert forward(o, lse) == 0
+        st = lib.fa2_get_device_status(sp, ctypes.byref(info))
+    finally:
+        lib.fa2_debug_forward_tag_skew(0)
+    assert st == FA2_ERR_CONFLICT, f"status {st}, site {info.value:#x}"
+    assert info.value == 0x10A
+
+    assert lib.fa2_clear_device_status() == 0
+    o2, lse2 = torch.empty_like(q), torch.empty_like(lse)
+    assert forward(o2, lse2) == 0
+    st = lib.fa2_get_device_status(sp, ctypes.byref(info))
+    assert st == 0, f"status {st} after clearing, site {info.value:#x}"
+    ro, rl = oracle_mod.attention_forward(t["q"], t["k"], t["v"], causal, scale)
+    where = f"after a conflict, B={B} H={H} N={N} d={d} causal={causal}"
     gh.check_o(gh.to_host_f64(o2), ro, where)
     gh.check_lse(lse2.cpu().numpy().astype(np.float64), rl, where)
