@@ -24,11 +24,6 @@
 
 namespace fa2 {
 
-// Heads per causal scheduling group of the main kernel (their Q, dO and dQ
-// accumulator stay in L2 while the group runs).
-#ifndef FA2_BWD_HEAD_GROUP
-#define FA2_BWD_HEAD_GROUP 16
-#endif
 
 // ------------------------------------------------------------- preprocess (B1)
 struct BwdPreParams {
@@ -204,7 +199,6 @@ struct BwdCfg {
   // d = 128 has no free columns left: dQ reuses the dP^T columns once dS is in smem
   static constexpr bool DQ_IN_DP = (D == 128);
   static constexpr uint32_t COL_DQ = DQ_IN_DP ? COL_DP : 256 + 2 * D;
-  static constexpr int HEAD_GROUP = FA2_BWD_HEAD_GROUP;  // heads per scheduling group
 };
 
 struct BwdParams {
@@ -220,6 +214,7 @@ struct BwdParams {
   int n_qtiles;           // query tiles: Np / 128
   int kq_offset;          // Nk - Nq: causal query i sees keys j <= i + kq_offset
   int causal;
+  int head_group;         // heads per causal scheduling group (see decode_item)
   float scale;
   float scale_log2;
 };
@@ -247,7 +242,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int u) {
 
 // Work item -> (key tile, batch*head). Non-causal items all cost the same: the
 // key tiles of one head are consecutive, so they run together and share the
-// head's Q/dO in L2. Causal items come in groups of HEAD_GROUP heads (their Q/dO
+// head's Q/dO in L2. Causal items come in groups of head_group heads (their Q/dO
 // stay in L2 while the group runs); inside a group the key tile is the slow
 // index, so the items with the most query blocks come first.
 __device__ __forceinline__ void decode_item(int item, int n_ktiles, int BH, int head_group,
@@ -406,7 +401,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         mbar_arrive(bar_item_full(n & 1));
         if (item < 0) break;
         int ktile, bh;
-        decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
+        decode_item(item, p.n_ktiles, p.BH, p.head_group, p.causal != 0, ktile, bh);
         const int i_first = qfirst(ktile);
         const int n_iter = steps_of(ktile);
         for (int it = 0; it < n_iter && ok; ++it, ++gs) {
@@ -488,7 +483,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const int item = take_item(n, 0x1209);
         if (item < 0) break;
         int ktile, bh;
-        decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
+        decode_item(item, p.n_ktiles, p.BH, p.head_group, p.causal != 0, ktile, bh);
         const int n_iter = steps_of(ktile);
         FA2_TRACE_AT(trace_cta, 40, n);
         ok = mbar_wait(bar_kv_full, n & 1, abort_flag, 0x1201) &&
@@ -605,7 +600,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const int item = take_item(n, 0x1709);
         if (item < 0) break;
         int ktile, bh;
-        decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
+        decode_item(item, p.n_ktiles, p.BH, p.head_group, p.causal != 0, ktile, bh);
         const int i_first = qfirst(ktile);
         const int n_iter = steps_of(ktile);
         for (int it = 0; WITH_DQ && it < n_iter; ++it) {
@@ -648,7 +643,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int item = take_item(n, 0x1309);
       if (item < 0) break;
       int ktile, bh;
-      decode_item(item, p.n_ktiles, p.BH, C::HEAD_GROUP, p.causal != 0, ktile, bh);
+      decode_item(item, p.n_ktiles, p.BH, p.head_group, p.causal != 0, ktile, bh);
       const int i_first = qfirst(ktile);
       const int n_iter = steps_of(ktile);
       FA2_TRACE_AT(trace_cta && threadIdx.x == 0, 44, n);

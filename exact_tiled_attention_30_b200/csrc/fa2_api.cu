@@ -182,6 +182,21 @@ fa2_status ensure_smem(KernelT kernel, int bytes, int dev, bool* done) {
 
 int sm_count(int dev);
 
+// Causal kernels walk their work in groups of heads, heaviest items first
+// inside a group, so that the tiles every item of a group re-reads stay in L2
+// while the group runs. The group is as many heads as fit a share of the
+// 126 MB L2 (at most 16): per head the forward re-reads K and V (4 N d bytes)
+// and the backward Q, dO and the fp32 dQ accumulator (8 N d bytes). Measured at
+// B=1 H=16 N=16384 d=128: 4 heads instead of 16 cut the backward's DRAM
+// traffic from 3.0 GB to 0.65 GB a launch (its algorithmic bytes: 0.67 GB) and
+// its time by 3 %; at N <= 4096 the group stays 16 heads, the fastest there.
+constexpr long long kL2GroupBudget = 64ll << 20;
+
+int causal_head_group(long long bytes_per_head) {
+  long long g = bytes_per_head > 0 ? kL2GroupBudget / bytes_per_head : 16;
+  return static_cast<int>(g < 1 ? 1 : (g > 16 ? 16 : g));
+}
+
 // Work-item counters of the persistent forward kernel. Each launch takes the
 // next slot of a ring (one per device) and a fresh nonzero 32-bit tag, and one
 // 32-bit memset on the launch's stream writes the tag into both halves of the
@@ -265,6 +280,7 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.BH = BH;
+  p.head_group = causal_head_group(4ll * Nk * D);
   fa2_status st = FA2_OK;
   p.counter = fwd_counter(dev, stream, &p.tag, &st);
   if (st != FA2_OK) return st;
@@ -367,6 +383,7 @@ fa2_status launch_bwd_main(const void* q, const void* k, const void* v, const vo
   bp.n_qtiles = w.Np / 128;
   bp.kq_offset = Nk - Nq;
   bp.causal = causal ? 1 : 0;
+  bp.head_group = causal_head_group(8ll * Nq * D);
   bp.scale = scale;
   bp.scale_log2 = scale * 1.4426950408889634f;
   // persistent: one CTA per SM (its shared memory allows no second one)

@@ -55,10 +55,6 @@
 
 namespace fa2 {
 
-// Heads per causal scheduling group (their K/V tiles stay in L2 while the group runs).
-#ifndef FA2_FWD_HEAD_GROUP
-#define FA2_FWD_HEAD_GROUP 16
-#endif
 
 template <int D>
 struct FwdCfg {
@@ -89,7 +85,6 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
   static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 of the largest P entry
-  static constexpr int HEAD_GROUP = FA2_FWD_HEAD_GROUP;    // causal launch order, see below
   // d = 64: one pair of weights in POLY_EVERY is exponentiated on the FMA pipe
   // (the MUFU unit is the tighter limit there; one in 8 measured fastest of
   // 2, 3, 4, 5, 6, 8, 12 and none); d = 128: MUFU only (measured faster)
@@ -111,13 +106,15 @@ struct FwdParams {
   int n_pairs;   // ceil(n_qtiles / 2)
   int BH;
   int causal;
+  int head_group;    // heads per causal scheduling group (see fwd_decode_item)
   float scale_log2;  // scale * log2(e)
 };
 
 // Work item -> (pair of query tiles, batch*head). Non-causal: the pairs of one
 // head are consecutive, so they run together and share its K/V tiles in L2.
-// Causal: groups of HEAD_GROUP heads (their K/V stay in L2 while the group
-// runs); inside a group the heaviest pairs of every head come first.
+// Causal: groups of head_group heads (their K/V stay in L2 while the group
+// runs; the host sizes the group to the L2); inside a group the heaviest pairs
+// of every head come first.
 __device__ __forceinline__ void fwd_decode_item(int item, int n_pairs, int BH, int head_group,
                                                 bool causal, int& pair, int& bh) {
   if (!causal) {
@@ -248,7 +245,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         mbar_arrive(bar_item_full(n & 1));
         if (item < 0) break;
         int pair, bh, n0, n1;
-        fwd_decode_item(item, p.n_pairs, p.BH, C::HEAD_GROUP, p.causal != 0, pair, bh);
+        fwd_decode_item(item, p.n_pairs, p.BH, p.head_group, p.causal != 0, pair, bh);
         tiles_of(pair, n0, n1);
         // Q0, Q1 once the previous item's S MMAs are done with the buffers
         if (n >= 1) ok = mbar_wait(bar_q_empty, (n - 1) & 1, abort_flag, 0x105);
@@ -334,7 +331,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const int item = take_item(n, 0x207);
         if (item < 0) break;
         int pair, bh, n0, n1;
-        fwd_decode_item(item, p.n_pairs, p.BH, C::HEAD_GROUP, p.causal != 0, pair, bh);
+        fwd_decode_item(item, p.n_pairs, p.BH, p.head_group, p.causal != 0, pair, bh);
         tiles_of(pair, n0, n1);
         FA2_TRACE_AT(trace_cta, 20, n);
         ok = mbar_wait(bar_q_full, n & 1, abort_flag, 0x201) && wait_kv(kg);
@@ -413,7 +410,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const int item = take_item(n, 0x306);
       if (item < 0) break;
       int pair, bh, n0, n1;
-      fwd_decode_item(item, p.n_pairs, p.BH, C::HEAD_GROUP, p.causal != 0, pair, bh);
+      fwd_decode_item(item, p.n_pairs, p.BH, p.head_group, p.causal != 0, pair, bh);
       tiles_of(pair, n0, n1);
       const int qt = 2 * pair + t;
       const int n_t = t ? n1 : n0;
