@@ -329,16 +329,19 @@ def grid_points():
 
 def run_grid(args):
     """One JSON line per grid point: forward, backward (three kernels) and their sum
-    in TFLOP/s on device-resident random bf16 inputs, CUDA events around `reps`
-    calls after warm-up (not the contract line; the contract line is the default
-    run)."""
+    in TFLOP/s on device-resident random bf16 inputs, CUDA events around enough
+    calls for at least ~60 ms of work (and at least 10) after warm-up, with the
+    nvidia-smi clocks sampled in that span (not the contract line; the contract
+    line is the default run)."""
     import torch
 
     import exact_tiled_attention_30_b200 as fa2
 
     fa2.load_library()
     peaks, _ = load_peaks()
-    reps = max(args.steps // 40, 5)
+    min_reps = max(args.steps // 40, 5)
+    visible = [e.strip() for e in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if e.strip()]
+    sampler = ClockSampler(visible[0] if visible else "0")
     for w in grid_points():
         if args.grid_filter and not any(f"{k}={w.get(k)}" in args.grid_filter.split(",")
                                         for k in ("d", "N")):
@@ -359,19 +362,27 @@ def run_grid(args):
             fa2.fa2_backward(q, k, v, o, lse, do, dq, dk, dv, causal, scale, ws)
 
         res = {}
+        t_in = []
         for name, fn in (("fwd", fwd), ("bwd", bwd)):
             for _ in range(args.warmup):
                 fn()
             torch.cuda.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            reps = int(min(2000, max(min_reps, math.ceil(60.0 / max(e0.elapsed_time(e1), 1e-3)))))
+            t_in.append(time.time())
+            e0.record()
             for _ in range(reps):
                 fn()
             e1.record()
             torch.cuda.synchronize()
+            t_in.append(time.time())
             res[name] = e0.elapsed_time(e1) / reps
         res["fwd+bwd"] = res["fwd"] + res["bwd"]
-        line = {"grid": True, **w}
+        line = {"grid": True, **w, "clocks": sampler.summary(t_in[0], t_in[-1])}
         for name, ms in res.items():
             tf = flops(w, name) / (ms * 1e-3) / 1e12
             line[name] = {"ms": round(ms, 4), "tflops": round(tf, 1),
@@ -379,6 +390,7 @@ def run_grid(args):
         print(json.dumps(line), flush=True)
         del q, k, v, do, o, lse, dq, dk, dv, ws
         torch.cuda.empty_cache()
+    sampler.stop()
 
 
 # --------------------------------------------------------------- GPU timing
