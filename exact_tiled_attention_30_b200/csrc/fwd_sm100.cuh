@@ -69,10 +69,10 @@ struct FwdCfg {
   static constexpr int OFF_K = 2 * TILE_BYTES;        // + s * 2 * TILE_BYTES
   static constexpr int OFF_V = 3 * TILE_BYTES;        // + s * 2 * TILE_BYTES
   static constexpr int OFF_BAR = TILE_BYTES * (2 + 2 * STAGES);
-  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2],
-  // o_free[2], drain, xmax[2 tiles][2 slots], xsum[2 tiles], item_full[2],
-  // item_empty[2]
-  static constexpr int NUM_BARS = 2 + 2 * STAGES + 9 + 6 + 4;
+  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2 tiles][2], p_full[2][2],
+  // o_done[2], o_free[2], drain, xmax[2 tiles][2 slots], xsum[2 tiles],
+  // item_full[2], item_empty[2], pv_done[2]
+  static constexpr int NUM_BARS = 2 + 2 * STAGES + 25;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;  // tmem slot, abort flag, items[2]
   // exchange between the two halves of a row: partial maxima [tile][slot][half][row]
   // and, at the end, partial sums [tile][half][l | lr][row]
@@ -83,7 +83,13 @@ struct FwdCfg {
   static constexpr int WARP_TMA = 16, WARP_MMA = 17;
   static constexpr int THREADS = 32 * 18;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  // d = 64 has room for three S buffers that the two query tiles take in turn
+  // (ROT, see the MMA issuer): S_t of the item's j-th key tile lives in buffer
+  // (2 j + t) mod 3, so each tile's next S is computed while its softmax runs.
+  // d = 128: one S buffer per tile.
+  static constexpr bool ROT = (D == 64);
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
+  static constexpr uint32_t COL_O0 = ROT ? 384 : 256, COL_O1 = ROT ? 448 : 256 + D;
   static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 of the largest P entry
   // d = 64: one pair of weights in POLY_EVERY is exponentiated on the FMA pipe
   // (the MUFU unit is the tighter limit there; one in 8 measured fastest of
@@ -163,15 +169,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   auto bar_kv_full = [&](int s) { return sbase + C::OFF_BAR + 8 * (2 + s); };
   auto bar_kv_empty = [&](int s) { return sbase + C::OFF_BAR + 8 * (2 + C::STAGES + s); };
   const uint32_t bar_base = sbase + C::OFF_BAR + 8 * (2 + 2 * C::STAGES);
-  auto bar_s_full = [&](int t) { return bar_base + 8 * t; };
-  auto bar_p_full = [&](int t) { return bar_base + 16 + 8 * t; };
-  auto bar_o_done = [&](int t) { return bar_base + 32 + 8 * t; };
-  auto bar_o_free = [&](int t) { return bar_base + 48 + 8 * t; };
-  const uint32_t bar_drain = bar_base + 64;
-  auto bar_xmax = [&](int t, int slot) { return bar_base + 72 + 16 * t + 8 * slot; };
-  auto bar_xsum = [&](int t) { return bar_base + 104 + 8 * t; };
-  auto bar_item_full = [&](int q) { return bar_base + 120 + 8 * q; };
-  auto bar_item_empty = [&](int q) { return bar_base + 136 + 8 * q; };
+  // s_full / p_full: d = 128 uses barrier 0 of each tile (phase = the tile's key
+  // tile count); d = 64 alternates barriers 0 and 1 (phase = count / 2), since
+  // its S runs two key tiles ahead of the softmax.
+  auto bar_s_full = [&](int t, int k) { return bar_base + 8 * (2 * t + k); };
+  auto bar_p_full = [&](int t, int k) { return bar_base + 32 + 8 * (2 * t + k); };
+  auto bar_o_done = [&](int t) { return bar_base + 64 + 8 * t; };
+  auto bar_o_free = [&](int t) { return bar_base + 80 + 8 * t; };
+  const uint32_t bar_drain = bar_base + 96;
+  auto bar_xmax = [&](int t, int slot) { return bar_base + 104 + 16 * t + 8 * slot; };
+  auto bar_xsum = [&](int t) { return bar_base + 136 + 8 * t; };
+  auto bar_item_full = [&](int q) { return bar_base + 152 + 8 * q; };
+  auto bar_item_empty = [&](int q) { return bar_base + 168 + 8 * q; };
+  auto bar_pv_done = [&](int t) { return bar_base + 184 + 8 * t; };  // d = 64: one phase per P V
+  // barrier index and phase parity of the g-th key tile of a query tile
+  auto sp_k = [&](int g) { return C::ROT ? (g & 1) : 0; };
+  auto sp_par = [&](int g) { return static_cast<uint32_t>(C::ROT ? ((g >> 1) & 1) : (g & 1)); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* item_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
@@ -184,8 +197,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       mbar_init(bar_kv_empty(s), 1);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(bar_s_full(t), 1);
-      mbar_init(bar_p_full(t), 256);
+      for (int k = 0; k < 2; ++k) {
+        mbar_init(bar_s_full(t, k), 1);
+        mbar_init(bar_p_full(t, k), 256);
+      }
+      mbar_init(bar_pv_done(t), 1);
       mbar_init(bar_o_done(t), 1);
       mbar_init(bar_o_free(t), 256);
       mbar_init(bar_xmax(t, 0), 256);
@@ -292,20 +308,29 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const SDesc dk0 = sdesc_make(sbase + C::OFF_K, 16, 1024);
       const SDesc dv0 = sdesc_make(sbase + C::OFF_V, C::CHUNK_BYTES, 1024);
       constexpr uint32_t STAGE16 = 2 * C::TILE_BYTES / 16;  // stage stride in descriptor units
-      auto issue_s = [&](int t, int g) {  // g: key tile counted over the CTA's items
+      // S buffer of tile t's j-th key tile of the current item
+      auto sbuf = [&](int t, int j) -> uint32_t {
+        if constexpr (C::ROT) return static_cast<uint32_t>((2 * j + t) % 3) * 128u;
+        return t ? C::COL_S1 : C::COL_S0;
+      };
+      int jt0 = 0, jt1 = 0;   // key tiles of query tile 0 / 1 so far (s_full, p_full phases)
+      // S_t of the item's key tile j, from the K/V ring slot of key tile g
+      // (counted over the CTA's items)
+      auto issue_s = [&](int t, int j, int g) {
         const uint32_t klo = dk0.lo + (g % C::STAGES) * STAGE16;
         const uint32_t qlo = t ? dq1.lo : dq0.lo;
-        const uint32_t dcol = tmem + (t ? C::COL_S1 : C::COL_S0);
+        const uint32_t dcol = tmem + sbuf(t, j);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = ((k >> 2) * C::CHUNK_BYTES + (k & 3) * 32) >> 4;
           umma_ss2(dcol, qlo + off, dq0.hi, klo + off, dk0.hi, IDESC_S, k > 0 ? 1u : 0u);
         }
-        umma_commit(bar_s_full(t));
+        const int gt = (t ? jt1 : jt0) + j;
+        umma_commit(bar_s_full(t, sp_k(gt)));
       };
-      auto issue_pv = [&](int t, int g, bool acc) {
+      auto issue_pv = [&](int t, int j, int g, bool acc) {
         const uint32_t vlo = dv0.lo + (g % C::STAGES) * STAGE16;
-        const uint32_t pcol = tmem + (t ? C::COL_S1 : C::COL_S0);
+        const uint32_t pcol = tmem + sbuf(t, j);
         const uint32_t ocol = tmem + (t ? C::COL_O1 : C::COL_O0);
         const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
@@ -315,10 +340,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           umma_ts2(ocol, pcol + k * 8 + (k >= 4 ? 32 : 0), vlo + k * (2048 >> 4), dv0.hi, IDESC_O,
                    k > 0 ? 1u : acc0);
         }
+        if constexpr (C::ROT) umma_commit(bar_pv_done(t));
+      };
+      auto wait_p = [&](int t, int j, unsigned int site) {
+        const int gt = (t ? jt1 : jt0) + j;
+        return mbar_wait(bar_p_full(t, sp_k(gt)), sp_par(gt), abort_flag, site);
       };
       bool ok = true;
       int kg = 0;             // key tiles consumed so far (K/V ring position)
-      int jt0 = 0, jt1 = 0;   // key tiles of query tile 0 / 1 so far (s_full, p_full phases)
       int kv_waited = -1;     // highest key tile (counted like kg) whose kv_full was waited for
       auto wait_kv = [&](int g) -> bool {
         if (g <= kv_waited) return true;
@@ -340,48 +369,97 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         tc_fence_after();
         // S of the item's first key tile: the S columns were last read by the
         // previous item's PV, which this thread issued before
-        issue_s(0, kg);
-        issue_s(1, kg);
+        issue_s(0, 0, kg);
+        issue_s(1, 0, kg);
         if (n1 == 1) umma_commit(bar_q_empty);  // every S of the item issued
-        for (int j = 0; j < n1 && ok; ++j) {
-          const int g = kg + j;
-          if (j < n0) {
-            ok = mbar_wait(bar_p_full(0), (jt0 + j) & 1, abort_flag, 0x204);
+        if constexpr (C::ROT) {
+          // Three S buffers: tile 0's S runs two key tiles ahead (S0_{j+2} takes
+          // the buffer P1_j leaves), tile 1's one (S1_{j+1} takes the buffer P0_j
+          // leaves), so both softmaxes find their next S ready when they finish.
+          // Issue order per key tile j: PV0_j, S1_{j+1}, PV1_j, S0_{j+2}.
+          if (n0 > 1) {
+            ok = wait_kv(kg + 1);
             if (!ok) break;
-            if (j == 0 && n > 0) {  // the epilogue of the previous item has read O0
-              ok = mbar_wait(bar_o_free(0), (n - 1) & 1, abort_flag, 0x208);
+            issue_s(0, 1, kg + 1);
+          }
+          for (int j = 0; j < n1 && ok; ++j) {
+            const int g = kg + j;
+            if (j < n0) {
+              ok = wait_p(0, j, 0x204);
+              if (!ok) break;
+              if (j == 0 && n > 0) {  // the epilogue of the previous item has read O0
+                ok = mbar_wait(bar_o_free(0), (n - 1) & 1, abort_flag, 0x208);
+                if (!ok) break;
+              }
+              FA2_TRACE_AT(trace_cta && n == 0, 16, j);
+              tc_fence_after();
+              issue_pv(0, j, g, j > 0);
+              if (j + 1 == n0) umma_commit(bar_o_done(0));
+              if (j + 1 < n1) {
+                ok = wait_kv(g + 1);
+                if (!ok) break;
+                issue_s(1, j + 1, g + 1);  // into the buffer PV0_j has just read
+                if (j + 2 == n1) umma_commit(bar_q_empty);  // the item's last S
+              }
+            }
+            ok = wait_p(1, j, 0x205);
+            if (!ok) break;
+            if (j == 0 && n > 0) {
+              ok = mbar_wait(bar_o_free(1), (n - 1) & 1, abort_flag, 0x209);
               if (!ok) break;
             }
-            FA2_TRACE_AT(trace_cta && n == 0, 16, j);
+            FA2_TRACE_AT(trace_cta && n == 0, 18, j);
             tc_fence_after();
-            issue_pv(0, g, j > 0);
-            if (j + 1 < n0) {
+            issue_pv(1, j, g, j > 0);
+            umma_commit(bar_kv_empty(g % C::STAGES));  // K and V of this key tile fully consumed
+            if (j + 1 == n1) umma_commit(bar_o_done(1));
+            if (j + 2 < n0) {
+              ok = wait_kv(g + 2);
+              if (!ok) break;
+              issue_s(0, j + 2, g + 2);  // into the buffer PV1_j has just read
+            }
+          }
+        } else {
+          for (int j = 0; j < n1 && ok; ++j) {
+            const int g = kg + j;
+            if (j < n0) {
+              ok = wait_p(0, j, 0x204);
+              if (!ok) break;
+              if (j == 0 && n > 0) {  // the epilogue of the previous item has read O0
+                ok = mbar_wait(bar_o_free(0), (n - 1) & 1, abort_flag, 0x208);
+                if (!ok) break;
+              }
+              FA2_TRACE_AT(trace_cta && n == 0, 16, j);
+              tc_fence_after();
+              issue_pv(0, j, g, j > 0);
+              if (j + 1 < n0) {
+                ok = wait_kv(g + 1);
+                if (!ok) break;
+                issue_s(0, j + 1, g + 1);  // overwrites S0/P0 after PV0 in issue order
+                FA2_TRACE_AT(trace_cta && n == 0, 17, j);
+              } else {
+                umma_commit(bar_o_done(0));
+              }
+            }
+            ok = wait_p(1, j, 0x205);
+            if (!ok) break;
+            if (j == 0 && n > 0) {
+              ok = mbar_wait(bar_o_free(1), (n - 1) & 1, abort_flag, 0x209);
+              if (!ok) break;
+            }
+            FA2_TRACE_AT(trace_cta && n == 0, 18, j);
+            tc_fence_after();
+            issue_pv(1, j, g, j > 0);
+            umma_commit(bar_kv_empty(g % C::STAGES));  // K and V of this key tile fully consumed
+            if (j + 1 < n1) {
               ok = wait_kv(g + 1);
               if (!ok) break;
-              issue_s(0, g + 1);  // overwrites S0/P0 after PV0 in issue order
-              FA2_TRACE_AT(trace_cta && n == 0, 17, j);
+              issue_s(1, j + 1, g + 1);
+              if (j + 2 == n1) umma_commit(bar_q_empty);  // the item's last S: Q no longer read
+              FA2_TRACE_AT(trace_cta && n == 0, 19, j);
             } else {
-              umma_commit(bar_o_done(0));
+              umma_commit(bar_o_done(1));
             }
-          }
-          ok = mbar_wait(bar_p_full(1), (jt1 + j) & 1, abort_flag, 0x205);
-          if (!ok) break;
-          if (j == 0 && n > 0) {
-            ok = mbar_wait(bar_o_free(1), (n - 1) & 1, abort_flag, 0x209);
-            if (!ok) break;
-          }
-          FA2_TRACE_AT(trace_cta && n == 0, 18, j);
-          tc_fence_after();
-          issue_pv(1, g, j > 0);
-          umma_commit(bar_kv_empty(g % C::STAGES));  // K and V of this key tile fully consumed
-          if (j + 1 < n1) {
-            ok = wait_kv(g + 1);
-            if (!ok) break;
-            issue_s(1, g + 1);
-            if (j + 2 == n1) umma_commit(bar_q_empty);  // the item's last S: Q no longer read
-            FA2_TRACE_AT(trace_cta && n == 0, 19, j);
-          } else {
-            umma_commit(bar_o_done(1));
           }
         }
         kg += n1;
@@ -398,7 +476,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int h = (warp >> 2) & 1;        // key half: keys [64h, 64h+64) of each tile
     const int row = threadIdx.x & 127;    // TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t scol = (t ? C::COL_S1 : C::COL_S0) + 64 * h;  // this half's scores
+    // this half's scores of the item's j-th key tile
+    auto scol_of = [&](int j) -> uint32_t {
+      if constexpr (C::ROT) return static_cast<uint32_t>((2 * j + t) % 3) * 128u + 64 * h;
+      return (t ? C::COL_S1 : C::COL_S0) + 64 * h;
+    };
     constexpr int DH = D / 2;                                    // O columns per half
     const uint32_t ocol = (t ? C::COL_O1 : C::COL_O0) + DH * h;
     float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX) + t * 512 + row;  // + slot*256 + half*128
@@ -426,7 +508,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       for (int j = 0; j < n_t; ++j) {
         const int jj = jt + j;
         FA2_TRACE_AT(trace_row, 8 * t + 0, j);
-        ok = mbar_wait(bar_s_full(t), jj & 1, abort_flag, 0x301);
+        ok = mbar_wait(bar_s_full(t, sp_k(jj)), sp_par(jj), abort_flag, 0x301);
         if (!ok) break;
         FA2_TRACE_AT(trace_row, 8 * t + 1, j);
         FA2_TRACE_AT(trace_item && j == 0, 25 + 4 * t, n);
@@ -436,6 +518,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const bool need_mask = (p.causal && j * C::BN + C::BN > qt * C::BM + 1 + p.kq_offset) ||
                                (j * C::BN + C::BN > p.Nk);
         const int lim = p.causal ? min(qrow + 1 + p.kq_offset, p.Nk) : p.Nk;  // keys [0, lim) allowed
+        const uint32_t scol = scol_of(j);
         float s[64];
         tmem_ld64(lane_base + scol, s);
         if (need_mask) {
@@ -518,9 +601,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         f2_split(rr2, rr_lo, rr_hi);
         l = l * alpha + (rs_lo + rs_hi);
         lr = lr * alpha + (rr_lo + rr_hi);
-        // O holds PV_0..PV_{j-1}: all complete, since S_j was issued after them.
+        // O must hold PV_0..PV_{j-1} complete. d = 128: it does, since S_j was
+        // issued after them. d = 64 (S runs ahead): wait for PV_{j-1} first.
         // Each half rescales its own D/2 columns of O.
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          if constexpr (C::ROT) {
+            ok = mbar_wait(bar_pv_done(t), static_cast<uint32_t>((jj - 1) & 1), abort_flag, 0x307);
+            if (!ok) break;
+            tc_fence_after();
+          }
 #pragma unroll 1
           for (int q = 0; q < DH / 32; ++q) {
             float o[32];
@@ -533,7 +622,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar_p_full(t));
+        mbar_arrive(bar_p_full(t, sp_k(jj)));
         FA2_TRACE_AT(trace_row, 8 * t + 4, j);
       }
       if (!ok) break;
