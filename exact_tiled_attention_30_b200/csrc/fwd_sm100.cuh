@@ -237,6 +237,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     mbar_arrive(bar_item_empty(n & 1));
     return item;
   };
+  // the same for the converged MMA warp, which counts as one consumer
+  auto take_item_w = [&](int n, int site) -> int {
+    if (!mbar_wait_all(bar_item_full(n & 1), (n >> 1) & 1, abort_flag, site)) return -1;
+    const int item = item_slot[n & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_item_empty(n & 1));
+    return item;
+  };
 
   if (warp == C::WARP_TMA) {
     // ------------------------------------------------- scheduler + TMA producer
@@ -299,7 +307,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     }
   } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop converged; elect.sync inside each MMA and
+    // commit picks the issuing lane (see umma_ss2_w).
+    {
       constexpr uint32_t IDESC_S = idesc_bf16(128, C::BN, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
       // descriptor halves of every operand buffer, built once
@@ -323,10 +333,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = ((k >> 2) * C::CHUNK_BYTES + (k & 3) * 32) >> 4;
-          umma_ss2(dcol, qlo + off, dq0.hi, klo + off, dk0.hi, IDESC_S, k > 0 ? 1u : 0u);
+          umma_ss2_w(dcol, qlo + off, dq0.hi, klo + off, dk0.hi, IDESC_S, k > 0 ? 1u : 0u);
         }
         const int gt = (t ? jt1 : jt0) + j;
-        umma_commit(bar_s_full(t, sp_k(gt)));
+        umma_commit_w(bar_s_full(t, sp_k(gt)));
       };
       auto issue_pv = [&](int t, int j, int g, bool acc) {
         const uint32_t vlo = dv0.lo + (g % C::STAGES) * STAGE16;
@@ -337,14 +347,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int k = 0; k < C::BN / 16; ++k) {
           // V: MN-major (d contiguous), 16 keys = 2 swizzle atoms of 8 rows. P of
           // keys [64h, 64h+64) sits in columns [64h, 64h+32)
-          umma_ts2(ocol, pcol + k * 8 + (k >= 4 ? 32 : 0), vlo + k * (2048 >> 4), dv0.hi, IDESC_O,
+          umma_ts2_w(ocol, pcol + k * 8 + (k >= 4 ? 32 : 0), vlo + k * (2048 >> 4), dv0.hi, IDESC_O,
                    k > 0 ? 1u : acc0);
         }
-        if constexpr (C::ROT) umma_commit(bar_pv_done(t));
+        if constexpr (C::ROT) umma_commit_w(bar_pv_done(t));
       };
       auto wait_p = [&](int t, int j, unsigned int site) {
         const int gt = (t ? jt1 : jt0) + j;
-        return mbar_wait(bar_p_full(t, sp_k(gt)), sp_par(gt), abort_flag, site);
+        return mbar_wait_all(bar_p_full(t, sp_k(gt)), sp_par(gt), abort_flag, site);
       };
       bool ok = true;
       int kg = 0;             // key tiles consumed so far (K/V ring position)
@@ -352,18 +362,18 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       auto wait_kv = [&](int g) -> bool {
         if (g <= kv_waited) return true;
         kv_waited = g;
-        if (!mbar_wait(bar_kv_full(g % C::STAGES), (g / C::STAGES) & 1, abort_flag, 0x203)) return false;
+        if (!mbar_wait_all(bar_kv_full(g % C::STAGES), (g / C::STAGES) & 1, abort_flag, 0x203)) return false;
         tc_fence_after();
         return true;
       };
       for (int n = 0; ok; ++n) {
-        const int item = take_item(n, 0x207);
+        const int item = take_item_w(n, 0x207);
         if (item < 0) break;
         int pair, bh, n0, n1;
         fwd_decode_item(item, p.n_pairs, p.BH, p.head_group, p.causal != 0, pair, bh);
         tiles_of(pair, n0, n1);
         FA2_TRACE_AT(trace_cta, 20, n);
-        ok = mbar_wait(bar_q_full, n & 1, abort_flag, 0x201) && wait_kv(kg);
+        ok = mbar_wait_all(bar_q_full, n & 1, abort_flag, 0x201) && wait_kv(kg);
         if (!ok) break;
         FA2_TRACE_AT(trace_cta, 21, n);
         tc_fence_after();
@@ -371,7 +381,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         // previous item's PV, which this thread issued before
         issue_s(0, 0, kg);
         issue_s(1, 0, kg);
-        if (n1 == 1) umma_commit(bar_q_empty);  // every S of the item issued
+        if (n1 == 1) umma_commit_w(bar_q_empty);  // every S of the item issued
         if constexpr (C::ROT) {
           // Three S buffers: tile 0's S runs two key tiles ahead (S0_{j+2} takes
           // the buffer P1_j leaves), tile 1's one (S1_{j+1} takes the buffer P0_j
@@ -388,36 +398,42 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               ok = wait_p(0, j, 0x204);
               if (!ok) break;
               if (j == 0 && n > 0) {  // the epilogue of the previous item has read O0
-                ok = mbar_wait(bar_o_free(0), (n - 1) & 1, abort_flag, 0x208);
+                ok = mbar_wait_all(bar_o_free(0), (n - 1) & 1, abort_flag, 0x208);
                 if (!ok) break;
               }
               FA2_TRACE_AT(trace_cta && n == 0, 16, j);
               tc_fence_after();
               issue_pv(0, j, g, j > 0);
-              if (j + 1 == n0) umma_commit(bar_o_done(0));
+              FA2_TRACE_AT(trace_cta && n == 0, 32, j);
+              if (j + 1 == n0) umma_commit_w(bar_o_done(0));
               if (j + 1 < n1) {
                 ok = wait_kv(g + 1);
                 if (!ok) break;
+                FA2_TRACE_AT(trace_cta && n == 0, 33, j);
                 issue_s(1, j + 1, g + 1);  // into the buffer PV0_j has just read
-                if (j + 2 == n1) umma_commit(bar_q_empty);  // the item's last S
+                if (j + 2 == n1) umma_commit_w(bar_q_empty);  // the item's last S
               }
+              FA2_TRACE_AT(trace_cta && n == 0, 17, j);
             }
             ok = wait_p(1, j, 0x205);
             if (!ok) break;
             if (j == 0 && n > 0) {
-              ok = mbar_wait(bar_o_free(1), (n - 1) & 1, abort_flag, 0x209);
+              ok = mbar_wait_all(bar_o_free(1), (n - 1) & 1, abort_flag, 0x209);
               if (!ok) break;
             }
             FA2_TRACE_AT(trace_cta && n == 0, 18, j);
             tc_fence_after();
             issue_pv(1, j, g, j > 0);
-            umma_commit(bar_kv_empty(g % C::STAGES));  // K and V of this key tile fully consumed
-            if (j + 1 == n1) umma_commit(bar_o_done(1));
+            FA2_TRACE_AT(trace_cta && n == 0, 35, j);
+            umma_commit_w(bar_kv_empty(g % C::STAGES));  // K and V of this key tile fully consumed
+            if (j + 1 == n1) umma_commit_w(bar_o_done(1));
             if (j + 2 < n0) {
               ok = wait_kv(g + 2);
               if (!ok) break;
+              FA2_TRACE_AT(trace_cta && n == 0, 36, j);
               issue_s(0, j + 2, g + 2);  // into the buffer PV1_j has just read
             }
+            FA2_TRACE_AT(trace_cta && n == 0, 19, j);
           }
         } else {
           for (int j = 0; j < n1 && ok; ++j) {
@@ -426,7 +442,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               ok = wait_p(0, j, 0x204);
               if (!ok) break;
               if (j == 0 && n > 0) {  // the epilogue of the previous item has read O0
-                ok = mbar_wait(bar_o_free(0), (n - 1) & 1, abort_flag, 0x208);
+                ok = mbar_wait_all(bar_o_free(0), (n - 1) & 1, abort_flag, 0x208);
                 if (!ok) break;
               }
               FA2_TRACE_AT(trace_cta && n == 0, 16, j);
@@ -438,27 +454,27 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 issue_s(0, j + 1, g + 1);  // overwrites S0/P0 after PV0 in issue order
                 FA2_TRACE_AT(trace_cta && n == 0, 17, j);
               } else {
-                umma_commit(bar_o_done(0));
+                umma_commit_w(bar_o_done(0));
               }
             }
             ok = wait_p(1, j, 0x205);
             if (!ok) break;
             if (j == 0 && n > 0) {
-              ok = mbar_wait(bar_o_free(1), (n - 1) & 1, abort_flag, 0x209);
+              ok = mbar_wait_all(bar_o_free(1), (n - 1) & 1, abort_flag, 0x209);
               if (!ok) break;
             }
             FA2_TRACE_AT(trace_cta && n == 0, 18, j);
             tc_fence_after();
             issue_pv(1, j, g, j > 0);
-            umma_commit(bar_kv_empty(g % C::STAGES));  // K and V of this key tile fully consumed
+            umma_commit_w(bar_kv_empty(g % C::STAGES));  // K and V of this key tile fully consumed
             if (j + 1 < n1) {
               ok = wait_kv(g + 1);
               if (!ok) break;
               issue_s(1, j + 1, g + 1);
-              if (j + 2 == n1) umma_commit(bar_q_empty);  // the item's last S: Q no longer read
+              if (j + 2 == n1) umma_commit_w(bar_q_empty);  // the item's last S: Q no longer read
               FA2_TRACE_AT(trace_cta && n == 0, 19, j);
             } else {
-              umma_commit(bar_o_done(1));
+              umma_commit_w(bar_o_done(1));
             }
           }
         }
@@ -467,7 +483,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         jt1 += n1;
       }
       // drain: every UMMA of this CTA has finished before TMEM is released
-      umma_commit(bar_drain);
+      umma_commit_w(bar_drain);
       mbar_drain_wait(bar_drain, 0, 0x206);
     }
   } else {
@@ -503,6 +519,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #ifdef FA2_TRACE
       const bool trace_row = trace_cta && n == 0 && row == 0 && h == 0;
       const bool trace_item = trace_cta && row == 0 && h == 0;
+      const bool trace_last = trace_cta && n == 0 && row == 96 && h == 1;  // last warp of the tile
 #endif
       FA2_TRACE_AT(trace_item, 24 + 4 * t, n);
       for (int j = 0; j < n_t; ++j) {
@@ -511,6 +528,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         ok = mbar_wait(bar_s_full(t, sp_k(jj)), sp_par(jj), abort_flag, 0x301);
         if (!ok) break;
         FA2_TRACE_AT(trace_row, 8 * t + 1, j);
+        FA2_TRACE_AT(trace_last, 8 * t + 5, j);
         FA2_TRACE_AT(trace_item && j == 0, 25 + 4 * t, n);
         tc_fence_after();
         const int k0 = j * C::BN + 64 * h;  // first key of this half
@@ -596,6 +614,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           tmem_st16(lane_base + scol + 16 * q, pk);
         }
         FA2_TRACE_AT(trace_row, 8 * t + 3, j);
+        FA2_TRACE_AT(trace_last, 8 * t + 6, j);
         float rs_lo, rs_hi, rr_lo, rr_hi;
         f2_split(rs2, rs_lo, rs_hi);
         f2_split(rr2, rr_lo, rr_hi);
@@ -624,6 +643,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         tc_fence_before();
         mbar_arrive(bar_p_full(t, sp_k(jj)));
         FA2_TRACE_AT(trace_row, 8 * t + 4, j);
+        FA2_TRACE_AT(trace_last, 8 * t + 7, j);
       }
       if (!ok) break;
       jt += n_t;
