@@ -374,6 +374,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_arrive(bar_item_empty(n & 1));
     return item;
   };
+  // the same for the converged MMA warp, which counts as one consumer
+  auto take_item_w = [&](int n, int site) -> int {
+    if (!mbar_wait_all(bar_item_full(n & 1), (n >> 1) & 1, abort_flag, site)) return -1;
+    const int item = item_slot[n & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_item_empty(n & 1));
+    return item;
+  };
   // causal: the first query tile that sees key tile ktile (query i sees keys
   // j <= i + kq_offset, the mask aligned to the bottom-right corner)
   auto qfirst = [&](int ktile) {
@@ -452,7 +460,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
   } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop converged; elect.sync inside each MMA and
+    // commit picks the issuing lane (see umma_ss2_w).
+    {
       constexpr uint32_t IDESC_SS = idesc_bf16(128, 128, false, false);   // S^T, dP^T
       constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);      // dV, dK
       constexpr uint32_t IDESC_QT = idesc_bf16(128, 128, true, true);     // dQ^T (d = 128)
@@ -473,21 +483,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const uint32_t qlo = dQk.lo + (g % C::STAGES) * TILE16;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_ss2(tmem + C::COL_S, dK.lo + kmaj(k), dK.hi, qlo + kmaj(k), dQk.hi, IDESC_SS,
+          umma_ss2_w(tmem + C::COL_S, dK.lo + kmaj(k), dK.hi, qlo + kmaj(k), dQk.hi, IDESC_SS,
                    k > 0 ? 1u : 0u);
-        umma_commit(bar_s_full);
+        umma_commit_w(bar_s_full);
       };
       bool ok = true;
       int gs = 0;
       for (int n = 0; ok; ++n) {
-        const int item = take_item(n, 0x1209);
+        const int item = take_item_w(n, 0x1209);
         if (item < 0) break;
         int ktile, bh;
         decode_item(item, p.n_ktiles, p.BH, p.head_group, p.causal != 0, ktile, bh);
         const int n_iter = steps_of(ktile);
         FA2_TRACE_AT(trace_cta, 40, n);
-        ok = mbar_wait(bar_kv_full, n & 1, abort_flag, 0x1201) &&
-             mbar_wait(bar_st_full(gs % C::STAGES), (gs / C::STAGES) & 1, abort_flag, 0x1202);
+        ok = mbar_wait_all(bar_kv_full, n & 1, abort_flag, 0x1201) &&
+             mbar_wait_all(bar_st_full(gs % C::STAGES), (gs / C::STAGES) & 1, abort_flag, 0x1202);
         if (!ok) break;
         FA2_TRACE_AT(trace_cta, 41, n);
         tc_fence_after();
@@ -500,26 +510,26 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           const uint32_t acc0 = it > 0 ? 1u : 0u;
           FA2_TRACE_AT(trace_cta && n == 0, 16, it);
           if (WITH_DQ && C::DQ_IN_DP && g > 0) {  // the dP^T columns hold dQ of step g-1 until read out
-            ok = mbar_wait(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1203);
+            ok = mbar_wait_all(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1203);
             if (!ok) break;
             tc_fence_after();
           }
           FA2_TRACE_AT(trace_cta && n == 0, 17, it);
           const int ds = g % C::DO_STAGES;
-          ok = mbar_wait(bar_do_full(ds), (g / C::DO_STAGES) & 1, abort_flag, 0x120B);
+          ok = mbar_wait_all(bar_do_full(ds), (g / C::DO_STAGES) & 1, abort_flag, 0x120B);
           if (!ok) break;
           tc_fence_after();
           const uint32_t dolo = dOk.lo + ds * TILE16;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)  // dP^T = V dO_i^T
-            umma_ss2(tmem + C::COL_DP, dV.lo + kmaj(k), dV.hi, dolo + kmaj(k), dOk.hi, IDESC_SS,
+            umma_ss2_w(tmem + C::COL_DP, dV.lo + kmaj(k), dV.hi, dolo + kmaj(k), dOk.hi, IDESC_SS,
                      k > 0 ? 1u : 0u);
-          umma_commit(bar_dp_full);
+          umma_commit_w(bar_dp_full);
           // dV += P^T dO_i once every group has written P^T
-          ok = mbar_wait(bar_p_ready, g & 1, abort_flag, 0x1204);
+          ok = mbar_wait_all(bar_p_ready, g & 1, abort_flag, 0x1204);
           if (!ok) break;
           if (it == 0 && n > 0) {  // the previous item's dK, dV have been read out
-            ok = mbar_wait(bar_dkv_free, (n - 1) & 1, abort_flag, 0x120A);
+            ok = mbar_wait_all(bar_dkv_free, (n - 1) & 1, abort_flag, 0x120A);
             if (!ok) break;
           }
           FA2_TRACE_AT(trace_cta && n == 0, 18, it);
@@ -529,19 +539,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           for (int k = 0; k < C::BM / 16; ++k) {
             // queries 16k..16k+15 sit in group g = 16k / CW at column CW g + (16k mod CW) / 2
             const uint32_t pcol = C::COL_S + C::CW * ((16 * k) / C::CW) + ((16 * k) % C::CW) / 2;
-            umma_ts2(tmem + C::COL_DV, tmem + pcol, domlo + k * (2048 >> 4), dOm.hi, IDESC_KV,
+            umma_ts2_w(tmem + C::COL_DV, tmem + pcol, domlo + k * (2048 >> 4), dOm.hi, IDESC_KV,
                      k > 0 ? 1u : acc0);
           }
-          umma_commit(bar_do_empty(ds));  // dV was the last reader of dO_i
+          umma_commit_w(bar_do_empty(ds));  // dV was the last reader of dO_i
           if (it + 1 < n_iter) {
-            ok = mbar_wait(bar_st_full((g + 1) % C::STAGES), ((g + 1) / C::STAGES) & 1, abort_flag,
+            ok = mbar_wait_all(bar_st_full((g + 1) % C::STAGES), ((g + 1) / C::STAGES) & 1, abort_flag,
                            0x1208);
             if (!ok) break;
             tc_fence_after();
             issue_s(g + 1);
           }
           // dK += dS^T Q_i and dQ once dS^T is in smem
-          ok = mbar_wait(bar_ds_ready, g & 1, abort_flag, 0x1205);
+          ok = mbar_wait_all(bar_ds_ready, g & 1, abort_flag, 0x1205);
           if (!ok) break;
           FA2_TRACE_AT(trace_cta && n == 0, 19, it);
           tc_fence_after();
@@ -549,7 +559,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             const uint32_t qmlo = dQm.lo + s * TILE16;
 #pragma unroll
             for (int k = 0; k < C::BM / 16; ++k)
-              umma_ss2(tmem + C::COL_DK, dSk.lo + kmaj(k), dSk.hi, qmlo + k * (2048 >> 4), dQm.hi,
+              umma_ss2_w(tmem + C::COL_DK, dSk.lo + kmaj(k), dSk.hi, qmlo + k * (2048 >> 4), dQm.hi,
                        IDESC_KV, k > 0 ? 1u : acc0);
           };
           // d = 128 issues dQ first: its drain gates the next step's dP, which
@@ -557,31 +567,31 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           if (!C::DQ_IN_DP) issue_dk();
           if constexpr (WITH_DQ) {
             if (!C::DQ_IN_DP && g > 0) {  // dQ of step g-1 must be read out before it is overwritten
-              ok = mbar_wait(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1206);
+              ok = mbar_wait_all(bar_dq_empty, (g - 1) & 1, abort_flag, 0x1206);
               if (!ok) break;
               tc_fence_after();
             }
   #pragma unroll
             for (int k = 0; k < C::BN / 16; ++k) {  // reduction over the 128 keys
               if (C::DQ_T)  // dQ^T = K^T dS^T
-                umma_ss2(tmem + C::COL_DQ, dKm.lo + k * (2048 >> 4), dKm.hi, dSm.lo + k * (2048 >> 4),
+                umma_ss2_w(tmem + C::COL_DQ, dKm.lo + k * (2048 >> 4), dKm.hi, dSm.lo + k * (2048 >> 4),
                          dSm.hi, IDESC_QT, k > 0 ? 1u : 0u);
               else  // dQ = dS K
-                umma_ss2(tmem + C::COL_DQ, dSm.lo + k * (2048 >> 4), dSm.hi, dKm.lo + k * (2048 >> 4),
+                umma_ss2_w(tmem + C::COL_DQ, dSm.lo + k * (2048 >> 4), dSm.hi, dKm.lo + k * (2048 >> 4),
                          dKm.hi, IDESC_Q, k > 0 ? 1u : 0u);
             }
-            umma_commit(bar_dq_full);
+            umma_commit_w(bar_dq_full);
           }
           if (C::DQ_IN_DP) issue_dk();
-          umma_commit(bar_dsm_free);
-          umma_commit(bar_st_empty(s));
+          umma_commit_w(bar_dsm_free);
+          umma_commit_w(bar_st_empty(s));
         }
         if (!ok) break;
-        umma_commit(bar_dkv_done);  // dK, dV of this item complete
-        umma_commit(bar_kv_empty);  // K_j, V_j no longer read
+        umma_commit_w(bar_dkv_done);  // dK, dV of this item complete
+        umma_commit_w(bar_kv_empty);  // K_j, V_j no longer read
         gs += n_iter;
       }
-      umma_commit(bar_drain);
+      umma_commit_w(bar_drain);
       mbar_drain_wait(bar_drain, 0, 0x1207);
     }
   } else if (warp == C::WARP_RED) {
@@ -1019,7 +1029,9 @@ __global__ void __launch_bounds__(BwdDqCfg<D>::THREADS, 1)
     }
   } else if (warp == C::WARP_MMA) {
     // --------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop converged; elect.sync inside each MMA and
+    // commit picks the issuing lane (see umma_ss2_w).
+    {
       constexpr uint32_t IDESC_SS = idesc_bf16(128, 128, false, false);  // S, dP
       constexpr uint32_t IDESC_DQ = idesc_bf16(128, D, false, true);     // dQ += dS K
       const SDesc dQk = sdesc_make(sbase + C::OFF_Q, 16, 1024);
@@ -1035,28 +1047,28 @@ __global__ void __launch_bounds__(BwdDqCfg<D>::THREADS, 1)
         const uint32_t vlo = dV.lo + (j % C::STAGES) * STAGE16;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_ss2(tmem + C::COL_S, dQk.lo + kmaj(k), dQk.hi, klo + kmaj(k), dK.hi, IDESC_SS,
+          umma_ss2_w(tmem + C::COL_S, dQk.lo + kmaj(k), dQk.hi, klo + kmaj(k), dK.hi, IDESC_SS,
                    k > 0 ? 1u : 0u);
-        umma_commit(bar_s_full);
+        umma_commit_w(bar_s_full);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_ss2(tmem + C::COL_DP, dOk.lo + kmaj(k), dOk.hi, vlo + kmaj(k), dV.hi, IDESC_SS,
+          umma_ss2_w(tmem + C::COL_DP, dOk.lo + kmaj(k), dOk.hi, vlo + kmaj(k), dV.hi, IDESC_SS,
                    k > 0 ? 1u : 0u);
-        umma_commit(bar_dp_full);
+        umma_commit_w(bar_dp_full);
       };
-      bool ok = mbar_wait(bar_q, 0, abort_flag, 0x1501) &&
-                mbar_wait(bar_kv_full(0), 0, abort_flag, 0x1502);
+      bool ok = mbar_wait_all(bar_q, 0, abort_flag, 0x1501) &&
+                mbar_wait_all(bar_kv_full(0), 0, abort_flag, 0x1502);
       if (ok) {
         tc_fence_after();
         issue_s_dp(0);
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         // the elementwise warps have read S_j and dP_j and written dS_j
-        ok = mbar_wait(bar_ds_ready, j & 1, abort_flag, 0x1503);
+        ok = mbar_wait_all(bar_ds_ready, j & 1, abort_flag, 0x1503);
         if (!ok) break;
         tc_fence_after();
         if (j + 1 < n_kv) {
-          ok = mbar_wait(bar_kv_full((j + 1) % C::STAGES), ((j + 1) / C::STAGES) & 1, abort_flag, 0x1504);
+          ok = mbar_wait_all(bar_kv_full((j + 1) % C::STAGES), ((j + 1) / C::STAGES) & 1, abort_flag, 0x1504);
           if (!ok) break;
           tc_fence_after();
           issue_s_dp(j + 1);
@@ -1064,13 +1076,13 @@ __global__ void __launch_bounds__(BwdDqCfg<D>::THREADS, 1)
         const uint32_t kmlo = dKm.lo + (j % C::STAGES) * STAGE16;
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k)  // dQ += dS_j K_j (reduction over keys)
-          umma_ss2(tmem + C::COL_DQ, dSk.lo + kmaj(k), dSk.hi, kmlo + k * (2048 >> 4), dKm.hi,
+          umma_ss2_w(tmem + C::COL_DQ, dSk.lo + kmaj(k), dSk.hi, kmlo + k * (2048 >> 4), dKm.hi,
                    IDESC_DQ, (j > 0 || k > 0) ? 1u : 0u);
-        umma_commit(bar_dsm_free);
-        umma_commit(bar_kv_empty(j % C::STAGES));
+        umma_commit_w(bar_dsm_free);
+        umma_commit_w(bar_kv_empty(j % C::STAGES));
       }
-      umma_commit(bar_dq_done);
-      umma_commit(bar_drain);
+      umma_commit_w(bar_dq_done);
+      umma_commit_w(bar_drain);
       mbar_drain_wait(bar_drain, 0, 0x1505);
     }
   } else {
