@@ -20,6 +20,7 @@
 //   3. fa2_bwd_dq_convert: dQ = bf16(scale * accumulator).
 #pragma once
 
+#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa2 {
@@ -184,6 +185,10 @@ struct BwdCfg {
   static constexpr int CW = 128 / NWG;                 // query columns per group
   static constexpr int WARP_TMA = 4 * NWG, WARP_MMA = 4 * NWG + 1, WARP_RED = 4 * NWG + 2;
   static constexpr int THREADS = 32 * (4 * NWG + 3);
+  // groups of 4 exponentials (of CW / 4 per thread and step) that P^T takes on
+  // the FMA pipe instead of MUFU: d = 128, 2 of 8 (measured +1-1.6 % over 0, 1
+  // and 3); d = 64, none (measured 1-3 % faster than 1, 2 or 3)
+  static constexpr int POLY_GROUPS = (D == 128) ? 2 : 0;
   static constexpr int ELEM_THREADS = 128 * NWG;
   // threads that stage dQ for the TMA reductions: d = 128, the warps whose
   // TMEM lanes (d rows of dQ^T) are [0, 64); d = 64, all (each group its own
@@ -667,18 +672,30 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // red.global. The TMEM columns are released as soon as the values are in
       // registers.
       const uint32_t stg = sbase + C::OFF_STG;
-      auto drain = [&](int it) -> bool {
+      // drain_ld: wait for dQ of step it, move this group's share into registers
+      // and release the TMEM columns; drain_st: send the registers on.
+      constexpr int DQW = C::DQ_T ? CW : D / C::NWG;
+      float dqv[DQW];
+      auto drain_ld = [&](int it) -> bool {
         if (!mbar_wait(bar_dq_full, (gs + it) & 1, abort_flag, 0x1304)) return false;
         FA2_TRACE_AT(trace_row, 8 * g + 4, it);
         tc_fence_after();
+        if constexpr (C::DQ_T) {
+          // lane r holds dQ^T[d = r][query CW g + q]
+          tmem_ld32(lane_base + C::COL_DQ + CW * g, dqv);
+        } else {
+          // lane r holds dQ[query r][d]; this group stages d columns [16 g, 16 g + 16)
+          static_assert(C::DQ_T || DQW == 16, "d = 64 stages all of dQ");
+          tmem_ld16(lane_base + C::COL_DQ + DQW * g, dqv);
+        }
+        tc_fence_before();
+        mbar_arrive(bar_dq_empty);
+        return true;
+      };
+      auto drain_st = [&](int it) -> bool {
         float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i_first + it) * C::BM) * D;
         const int gg = gs + it;
         if constexpr (C::DQ_T) {
-          // lane r holds dQ^T[d = r][query CW g + q]
-          float v[CW];
-          tmem_ld32(lane_base + C::COL_DQ + CW * g, v);
-          tc_fence_before();
-          mbar_arrive(bar_dq_empty);
           if (r < 64) {
             // staged: row q of box r/32 holds query CW g + q; d = r sits in 16-byte
             // unit ((r mod 32) / 4) xor (row mod 8) of the 128-byte swizzle. This is
@@ -690,7 +707,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
             for (int q = 0; q < CW; ++q) {
               const int row = CW * g + q;
-              st_shared_f32(box + row * 128 + ((unit ^ (row & 7)) << 4) + word, v[q]);
+              st_shared_f32(box + row * 128 + ((unit ^ (row & 7)) << 4) + word, dqv[q]);
             }
             fence_async_smem();
             mbar_arrive(bar_staged);
@@ -698,24 +715,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             // each warp instruction adds 32 consecutive d values of one query row
             float* col = acc + static_cast<size_t>(CW * g) * D + r;
 #pragma unroll
-            for (int q = 0; q < CW; ++q) red_add(col + static_cast<size_t>(q) * D, v[q]);
+            for (int q = 0; q < CW; ++q) red_add(col + static_cast<size_t>(q) * D, dqv[q]);
           }
         } else {
-          // lane r holds dQ[query r][d]; this group stages d columns [16 g, 16 g + 16)
-          constexpr int DW = D / C::NWG;
-          static_assert(DW == 16, "d = 64 stages all of dQ");
-          float v[DW];
-          tmem_ld16(lane_base + C::COL_DQ + DW * g, v);
-          tc_fence_before();
-          mbar_arrive(bar_dq_empty);
           if (gg + n > 0 && !mbar_wait(bar_stg_free, (gg + n - 1) & 1, abort_flag, 0x1306)) return false;
 #pragma unroll
-          for (int u = 0; u < DW / 4; ++u) {
-            const int col = DW * g + 4 * u;
+          for (int u = 0; u < DQW / 4; ++u) {
+            const int col = DQW * g + 4 * u;
             const uint32_t box = stg + (col >> 5) * C::STG_BOX_BYTES;
             const uint32_t unit = static_cast<uint32_t>((col & 31) >> 2);
-            st_shared_v4(box + r * 128 + ((unit ^ (r & 7)) << 4), v[4 * u], v[4 * u + 1], v[4 * u + 2],
-                         v[4 * u + 3]);
+            st_shared_v4(box + r * 128 + ((unit ^ (r & 7)) << 4), dqv[4 * u], dqv[4 * u + 1], dqv[4 * u + 2],
+                         dqv[4 * u + 3]);
           }
           fence_async_smem();
           mbar_arrive(bar_staged);
@@ -723,6 +733,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         FA2_TRACE_AT(trace_row, 8 * g + 5, it);
         return true;
       };
+      auto drain = [&](int it) -> bool { return drain_ld(it) && drain_st(it); };
       for (int it = 0; it < n_iter; ++it) {
         const int i = i_first + it;
         const int gg = gs + it;
@@ -754,7 +765,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             float x0, x1, x2, x3;
             f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
             f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
-            float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            float p0, p1, p2, p3;
+            if (e / 4 < C::POLY_GROUPS) {  // FMA pipe: takes load off the MUFU unit
+              exp2_poly2(x0, x1, p0, p1);
+              exp2_poly2(x2, x3, p2, p3);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+              p2 = ex2(x2);
+              p3 = ex2(x3);
+            }
             if (diag) {  // query i*128 + q sees key ktile*128 + r only if r <= q + off
               const int q = CW * g + e;
               if (q + off < r) p0 = 0.f;
@@ -780,6 +800,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         // dS^T = P^T (dP^T - D) for the same columns, bf16 into the swizzled smem tile
         ok = mbar_wait(bar_dp_full, gg & 1, abort_flag, 0x1302);
         if (!ok) break;
+        FA2_TRACE_AT(trace_row, 8 * g + 6, it);
         tc_fence_after();
         uint32_t dk[CW / 2];
         {
@@ -807,6 +828,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           ok = mbar_wait(bar_dsm_free, (gg - 1) & 1, abort_flag, 0x1303);
           if (!ok) break;
         }
+        FA2_TRACE_AT(trace_row, 8 * g + 7, it);
 #pragma unroll
         for (int u = 0; u < CW / 8; ++u) {
           const uint32_t off = sw128_offset(r, (CW / 8) * g + u);

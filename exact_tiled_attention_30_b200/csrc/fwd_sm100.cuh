@@ -529,6 +529,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         if (!ok) break;
         FA2_TRACE_AT(trace_row, 8 * t + 1, j);
         FA2_TRACE_AT(trace_last, 8 * t + 5, j);
+        FA2_TRACE_AT(trace_cta && n == 0 && t == 0 && (threadIdx.x & 31) == 0, 56 + warp, j);
         FA2_TRACE_AT(trace_item && j == 0, 25 + 4 * t, n);
         tc_fence_after();
         const int k0 = j * C::BN + 64 * h;  // first key of this half
@@ -644,6 +645,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         mbar_arrive(bar_p_full(t, sp_k(jj)));
         FA2_TRACE_AT(trace_row, 8 * t + 4, j);
         FA2_TRACE_AT(trace_last, 8 * t + 7, j);
+        FA2_TRACE_AT(trace_cta && n == 0 && (threadIdx.x & 31) == 0, 40 + warp, j);
       }
       if (!ok) break;
       jt += n_t;
