@@ -19,13 +19,16 @@
 //                 other warps through a two-slot ring, loads Q0, Q1 once the
 //                 previous item's last S MMA is done, K_j/V_j into a STAGES-deep
 //                 ring that continues across items
-//   warp 17       MMA issuer + TMEM owner. Per key tile j it issues
-//                 PV0_j, S0_{j+1}, PV1_j, S1_{j+1} (in that order), so while one
-//                 tile's softmax runs the tensor core works on the other tile:
-//                 S_t = Q_t K_j^T (smem x smem -> TMEM) and O_t += P_t V_j (P from
-//                 TMEM, V from smem). The single issue order also keeps the two
-//                 tiles' softmax phases apart (measured: one issuer per tile let
-//                 them drift into step and contend for the MUFU unit).
+//   warp 17       MMA issuer + TMEM owner, running converged (elect.sync
+//                 inside each MMA picks the lane). Per key tile j it issues
+//                 PV0_j, S0_{j+1}, PV1_j, S1_{j+1} at d = 128 and PV0_j,
+//                 S1_{j+1}, PV1_j, S0_{j+2} at d = 64 (three rotating S
+//                 buffers), so while one tile's softmax runs the tensor core
+//                 works on the other tile: S_t = Q_t K_j^T (smem x smem -> TMEM)
+//                 and O_t += P_t V_j (P from TMEM, V from smem). The single issue
+//                 order also keeps the two tiles' softmax phases apart (measured:
+//                 one issuer per tile let them drift into step and contend for
+//                 the MUFU unit).
 //   warps 0-7     softmax of query tile 0, warps 8-15 of query tile 1. Two
 //                 warpgroups per tile split each row: warpgroup h owns keys
 //                 [64h, 64h+64) of row r (TMEM lane r): tcgen05.ld of its 64
@@ -37,8 +40,9 @@
 //                 O / l, stored with lanes transposed in groups so that every
 //                 store instruction writes whole row segments; O is released to
 //                 the next item's first PV as soon as it has been read.
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
-// O1 [256+D, 256+2D). Scores are kept in base 2: c = scale * log2(e) folds the
+// Tensor memory (512 columns): d = 128: S0 [0,128), S1 [128,256), O0 [256,384),
+// O1 [384,512); d = 64: S buffers [0,128), [128,256), [256,384), O0 [384,448),
+// O1 [448,512). Scores are kept in base 2: c = scale * log2(e) folds the
 // softmax scale into the exponent and m is stored pre-multiplied by c.
 //
 // Rescaling: a row's reference max m only moves when the new tile's max exceeds
