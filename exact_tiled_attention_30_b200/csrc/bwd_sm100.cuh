@@ -397,7 +397,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 
   if (warp == C::WARP_TMA) {
     // --------------------------------------------------- scheduler + TMA producer
-    if (lane == 0) {
+    // The whole warp runs this loop converged; elect.sync inside each copy and
+    // expect_tx picks the issuing lane (see umma_ss2_w).
+    {
       int last_st_parity[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) last_st_parity[s] = -1;
       int last_do_parity[C::DO_STAGES];
@@ -406,12 +408,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       bool ok = true;
       int gs = 0;
       for (int n = 0; ok; ++n) {
-        int item = static_cast<int>(atomicAdd(p.counter, 1u));
+        int item = 0;
+        if (lane == 0) item = static_cast<int>(atomicAdd(p.counter, 1u));
+        item = __shfl_sync(0xffffffffu, item, 0);
         if (item >= n_items) item = -1;
-        if (n >= 2) ok = mbar_wait(bar_item_empty(n & 1), ((n >> 1) - 1) & 1, abort_flag, 0x1100);
+        if (n >= 2) ok = mbar_wait_all(bar_item_empty(n & 1), ((n >> 1) - 1) & 1, abort_flag, 0x1100);
         if (!ok) break;
-        item_slot[n & 1] = item;
-        mbar_arrive(bar_item_full(n & 1));
+        if (lane == 0) {
+          item_slot[n & 1] = item;
+          mbar_arrive(bar_item_full(n & 1));
+        }
+        __syncwarp();
         if (item < 0) break;
         int ktile, bh;
         decode_item(item, p.n_ktiles, p.BH, p.head_group, p.causal != 0, ktile, bh);
@@ -420,38 +427,41 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int it = 0; it < n_iter && ok; ++it, ++gs) {
           const int i = i_first + it;
           const int s = gs % C::STAGES;
-          if (gs >= C::STAGES) ok = mbar_wait(bar_st_empty(s), ((gs / C::STAGES) - 1) & 1, abort_flag, 0x1101);
+          FA2_TRACE_AT(trace_cta && n == 0, 54, it);
+          if (gs >= C::STAGES) ok = mbar_wait_all(bar_st_empty(s), ((gs / C::STAGES) - 1) & 1, abort_flag, 0x1101);
           if (!ok) break;
+          FA2_TRACE_AT(trace_cta && n == 0, 52, it);
           if (it == 1 || n_iter == 1) {
             // K_j, V_j (after the first step's Q/dO is on its way) once the
             // previous item's MMAs are done with the buffers
-            if (n >= 1) ok = mbar_wait(bar_kv_empty, (n - 1) & 1, abort_flag, 0x1104);
+            if (n >= 1) ok = mbar_wait_all(bar_kv_empty, (n - 1) & 1, abort_flag, 0x1104);
             if (!ok) break;
-            mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE_BYTES);
+            mbar_arrive_expect_tx_w(bar_kv_full, 2 * C::TILE_BYTES);
             for (int c = 0; c < C::CHUNKS; ++c) {
-              tma_load_3d(sbase + C::OFF_K + c * C::CHUNK_BYTES, &tm_k, bar_kv_full, c * 64, ktile * C::BN, bh);
-              tma_load_3d(sbase + C::OFF_V + c * C::CHUNK_BYTES, &tm_v, bar_kv_full, c * 64, ktile * C::BN, bh);
+              tma_load_3d_w(sbase + C::OFF_K + c * C::CHUNK_BYTES, &tm_k, bar_kv_full, c * 64, ktile * C::BN, bh);
+              tma_load_3d_w(sbase + C::OFF_V + c * C::CHUNK_BYTES, &tm_v, bar_kv_full, c * 64, ktile * C::BN, bh);
             }
             last_kv_parity = n & 1;
           }
           const uint32_t bar = bar_st_full(s);
-          mbar_arrive_expect_tx(bar, C::TILE_BYTES + 2 * C::VEC_BYTES);
+          mbar_arrive_expect_tx_w(bar, C::TILE_BYTES + 2 * C::VEC_BYTES);
           for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_3d(sbase + C::OFF_Q + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar,
+            tma_load_3d_w(sbase + C::OFF_Q + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar,
                         c * 64, i * C::BM, bh);
           const size_t voff = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * C::BM;
           const uint32_t vec = sbase + C::OFF_VEC + s * 2 * C::VEC_BYTES;
-          bulk_load(vec, p.lse2 + voff, C::VEC_BYTES, bar);
-          bulk_load(vec + C::VEC_BYTES, p.delta + voff, C::VEC_BYTES, bar);
+          bulk_load_w(vec, p.lse2 + voff, C::VEC_BYTES, bar);
+          bulk_load_w(vec + C::VEC_BYTES, p.delta + voff, C::VEC_BYTES, bar);
+          FA2_TRACE_AT(trace_cta && n == 0, 53, it);
           last_st_parity[s] = (gs / C::STAGES) & 1;
           // dO_i once dV of the step that last used this dO buffer is done
           const int ds = gs % C::DO_STAGES;
           if (gs >= C::DO_STAGES)
-            ok = mbar_wait(bar_do_empty(ds), ((gs / C::DO_STAGES) - 1) & 1, abort_flag, 0x1105);
+            ok = mbar_wait_all(bar_do_empty(ds), ((gs / C::DO_STAGES) - 1) & 1, abort_flag, 0x1105);
           if (!ok) break;
-          mbar_arrive_expect_tx(bar_do_full(ds), C::TILE_BYTES);
+          mbar_arrive_expect_tx_w(bar_do_full(ds), C::TILE_BYTES);
           for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_3d(sbase + C::OFF_DO + ds * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do,
+            tma_load_3d_w(sbase + C::OFF_DO + ds * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do,
                         bar_do_full(ds), c * 64, i * C::BM, bh);
           last_do_parity[ds] = (gs / C::DO_STAGES) & 1;
         }
@@ -549,9 +559,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           }
           umma_commit_w(bar_do_empty(ds));  // dV was the last reader of dO_i
           if (it + 1 < n_iter) {
+            FA2_TRACE_AT(trace_cta && n == 0, 50, it);
             ok = mbar_wait_all(bar_st_full((g + 1) % C::STAGES), ((g + 1) / C::STAGES) & 1, abort_flag,
                            0x1208);
             if (!ok) break;
+            FA2_TRACE_AT(trace_cta && n == 0, 51, it);
             tc_fence_after();
             issue_s(g + 1);
           }
@@ -744,6 +756,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         // LSE2 and D of this query block were written by the TMA (async proxy)
         ok = mbar_wait(bar_st_full(s), (gg / C::STAGES) & 1, abort_flag, 0x1300);
         if (!ok) break;
+        FA2_TRACE_AT(trace_row, 48 + g, it);
         ok = mbar_wait(bar_s_full, gg & 1, abort_flag, 0x1301);
         if (!ok) break;
         FA2_TRACE_AT(trace_row, 8 * g + 1, it);

@@ -252,55 +252,63 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   if (warp == C::WARP_TMA) {
     // ------------------------------------------------- scheduler + TMA producer
-    if (lane == 0) {
+    // The whole warp runs this loop converged; elect.sync inside each copy and
+    // expect_tx picks the issuing lane (see umma_ss2_w).
+    {
       int last_parity[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) last_parity[s] = -1;
       int last_q_parity = -1;
       bool ok = true;
       int kg = 0;  // key tiles loaded so far
       for (int n = 0; ok; ++n) {
-        const unsigned long long v = atomicAdd(p.counter, 1ull);
         int item = -1;
-        if (static_cast<unsigned int>(v >> 32) != p.tag) {
-          report_conflict(0x10A);  // the slot now belongs to another launch: stop
-        } else {
-          const unsigned int taken = static_cast<unsigned int>(v) - p.tag;
-          if (taken < static_cast<unsigned int>(n_items)) item = static_cast<int>(taken);
+        if (lane == 0) {
+          const unsigned long long v = atomicAdd(p.counter, 1ull);
+          if (static_cast<unsigned int>(v >> 32) != p.tag) {
+            report_conflict(0x10A);  // the slot now belongs to another launch: stop
+          } else {
+            const unsigned int taken = static_cast<unsigned int>(v) - p.tag;
+            if (taken < static_cast<unsigned int>(n_items)) item = static_cast<int>(taken);
+          }
         }
-        if (n >= 2) ok = mbar_wait(bar_item_empty(n & 1), ((n >> 1) - 1) & 1, abort_flag, 0x104);
+        item = __shfl_sync(0xffffffffu, item, 0);
+        if (n >= 2) ok = mbar_wait_all(bar_item_empty(n & 1), ((n >> 1) - 1) & 1, abort_flag, 0x104);
         if (!ok) break;
-        item_slot[n & 1] = item;
-        mbar_arrive(bar_item_full(n & 1));
+        if (lane == 0) {
+          item_slot[n & 1] = item;
+          mbar_arrive(bar_item_full(n & 1));
+        }
+        __syncwarp();
         if (item < 0) break;
         int pair, bh, n0, n1;
         fwd_decode_item(item, p.n_pairs, p.BH, p.head_group, p.causal != 0, pair, bh);
         tiles_of(pair, n0, n1);
         // Q0, Q1 once the previous item's S MMAs are done with the buffers
-        if (n >= 1) ok = mbar_wait(bar_q_empty, (n - 1) & 1, abort_flag, 0x105);
+        if (n >= 1) ok = mbar_wait_all(bar_q_empty, (n - 1) & 1, abort_flag, 0x105);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar_q_full, 2 * C::TILE_BYTES);
+        mbar_arrive_expect_tx_w(bar_q_full, 2 * C::TILE_BYTES);
         for (int c = 0; c < C::CHUNKS; ++c) {
-          tma_load_3d(sbase + C::OFF_Q + c * C::CHUNK_BYTES, &tm_q, bar_q_full, c * 64,
+          tma_load_3d_w(sbase + C::OFF_Q + c * C::CHUNK_BYTES, &tm_q, bar_q_full, c * 64,
                       2 * pair * C::BM, bh);
-          tma_load_3d(sbase + C::OFF_Q + C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar_q_full,
+          tma_load_3d_w(sbase + C::OFF_Q + C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bar_q_full,
                       c * 64, (2 * pair + 1) * C::BM, bh);
         }
         last_q_parity = n & 1;
         for (int j = 0; j < n1 && ok; ++j, ++kg) {
           const int s = kg % C::STAGES;
           const int u = kg / C::STAGES;
-          if (u > 0) ok = mbar_wait(bar_kv_empty(s), (u - 1) & 1, abort_flag, 0x101);
+          if (u > 0) ok = mbar_wait_all(bar_kv_empty(s), (u - 1) & 1, abort_flag, 0x101);
           if (!ok) break;
 #ifdef FA2_TEST_HOOKS
           if (g_test_stall_kv > 0 && kg + 1 == g_test_stall_kv) continue;  // planted stall
 #endif
           const uint32_t kdst = sbase + C::OFF_K + s * 2 * C::TILE_BYTES;
           const uint32_t vdst = sbase + C::OFF_V + s * 2 * C::TILE_BYTES;
-          mbar_arrive_expect_tx(bar_kv_full(s), 2 * C::TILE_BYTES);
+          mbar_arrive_expect_tx_w(bar_kv_full(s), 2 * C::TILE_BYTES);
           for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_3d(kdst + c * C::CHUNK_BYTES, &tm_k, bar_kv_full(s), c * 64, j * C::BN, bh);
+            tma_load_3d_w(kdst + c * C::CHUNK_BYTES, &tm_k, bar_kv_full(s), c * 64, j * C::BN, bh);
           for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_3d(vdst + c * C::CHUNK_BYTES, &tm_v, bar_kv_full(s), c * 64, j * C::BN, bh);
+            tma_load_3d_w(vdst + c * C::CHUNK_BYTES, &tm_v, bar_kv_full(s), c * 64, j * C::BN, bh);
           last_parity[s] = u & 1;
         }
       }
