@@ -771,6 +771,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         {
           float sv[CW];
           tmem_ld32(lane_base + C::COL_S + CW * g, sv);
+          FA2_TRACE_AT(trace_row, 56 + g, it);
           const unsigned long long c2 = f2(c, c);
           // keys past query q + off are masked; off >= 127 masks none
           const int off = i * C::BM + p.kq_offset - ktile * C::BN;
@@ -804,6 +805,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           }
         }
         // P^T over the group's own first CW/2 S^T columns (already read above)
+        FA2_TRACE_AT(trace_row, 58 + g, it);
         tmem_st16(lane_base + C::COL_S + CW * g, pk);
         tmem_wait_st();
         tc_fence_before();

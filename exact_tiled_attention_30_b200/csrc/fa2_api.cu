@@ -257,11 +257,23 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
                           int H, int Nq, int Nk, int causal, float scale, cudaStream_t stream,
                           int dev) {
   using C = FwdCfg<D>;
+  // d = 128 without the causal mask: the instantiation that starts each item's
+  // tile 0 while the previous item's tile 1 finishes (every item's two query
+  // tiles then have the same number of key tiles)
+  const bool early = (D == 128) && !causal;
   static bool smem_set[kMaxDevices] = {false};
+  static bool smem_set_early[kMaxDevices] = {false};
+  (void)smem_set_early;
+  (void)early;
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lock(mu);
-    fa2_status st = ensure_smem(fa2::fa2_fwd_kernel<D>, C::SMEM_ALLOC, dev, smem_set);
+    fa2_status st;
+    if constexpr (D == 128)
+      st = early ? ensure_smem(fa2::fa2_fwd_kernel<D, true>, C::SMEM_ALLOC, dev, smem_set_early)
+                 : ensure_smem(fa2::fa2_fwd_kernel<D, false>, C::SMEM_ALLOC, dev, smem_set);
+    else
+      st = ensure_smem(fa2::fa2_fwd_kernel<D, false>, C::SMEM_ALLOC, dev, smem_set);
     if (st != FA2_OK) return st;
   }
   const int BH = B * H;
@@ -287,7 +299,14 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
   // persistent: one CTA per SM (its shared memory and TMEM allow no second one)
   const long long items = static_cast<long long>(BH) * p.n_pairs;
   const int ctas = static_cast<int>(items < sm_count(dev) ? items : sm_count(dev));
-  fa2::fa2_fwd_kernel<D><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  if constexpr (D == 128) {
+    if (early)
+      fa2::fa2_fwd_kernel<D, true><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    else
+      fa2::fa2_fwd_kernel<D, false><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  } else {
+    fa2::fa2_fwd_kernel<D, false><<<ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  }
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
   return FA2_OK;
 }
