@@ -20,6 +20,8 @@
 //   3. fa2_bwd_dq_convert: dQ = bf16(scale * accumulator).
 #pragma once
 
+#include <type_traits>
+
 #include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
 
@@ -776,33 +778,42 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           // keys past query q + off are masked; off >= 127 masks none
           const int off = i * C::BM + p.kq_offset - ktile * C::BN;
           const bool diag = p.causal && off < C::BN - 1;
+          // the same loop twice, with and without the causal mask, so that the
+          // common (unmasked) case has no branch between its independent groups
+          auto form_p = [&](auto masked) {
 #pragma unroll
-          for (int e = 0; e < CW; e += 4) {
-            const float4 l4 = make_float4(lds_f32(lse2 + e), lds_f32(lse2 + e + 1), lds_f32(lse2 + e + 2),
-                                          lds_f32(lse2 + e + 3));
-            float x0, x1, x2, x3;
-            f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
-            f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
-            float p0, p1, p2, p3;
-            if (e / 4 < C::POLY_GROUPS) {  // FMA pipe: takes load off the MUFU unit
-              exp2_poly2(x0, x1, p0, p1);
-              exp2_poly2(x2, x3, p2, p3);
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
-              p2 = ex2(x2);
-              p3 = ex2(x3);
+            for (int e = 0; e < CW; e += 4) {
+              const float4 l4 = make_float4(lds_f32(lse2 + e), lds_f32(lse2 + e + 1), lds_f32(lse2 + e + 2),
+                                            lds_f32(lse2 + e + 3));
+              float x0, x1, x2, x3;
+              f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
+              f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
+              float p0, p1, p2, p3;
+              if (e / 4 < C::POLY_GROUPS) {  // FMA pipe: takes load off the MUFU unit
+                exp2_poly2(x0, x1, p0, p1);
+                exp2_poly2(x2, x3, p2, p3);
+              } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+                p2 = ex2(x2);
+                p3 = ex2(x3);
+              }
+              if constexpr (decltype(masked)::value) {
+                // query i*128 + q sees key ktile*128 + r only if r <= q + off
+                const int q = CW * g + e;
+                p0 = q + off < r ? 0.f : p0;
+                p1 = q + 1 + off < r ? 0.f : p1;
+                p2 = q + 2 + off < r ? 0.f : p2;
+                p3 = q + 3 + off < r ? 0.f : p3;
+              }
+              pk[e / 2] = pack_bf16(p0, p1);
+              pk[e / 2 + 1] = pack_bf16(p2, p3);
             }
-            if (diag) {  // query i*128 + q sees key ktile*128 + r only if r <= q + off
-              const int q = CW * g + e;
-              if (q + off < r) p0 = 0.f;
-              if (q + 1 + off < r) p1 = 0.f;
-              if (q + 2 + off < r) p2 = 0.f;
-              if (q + 3 + off < r) p3 = 0.f;
-            }
-            pk[e / 2] = pack_bf16(p0, p1);
-            pk[e / 2 + 1] = pack_bf16(p2, p3);
-          }
+          };
+          if (diag)
+            form_p(std::integral_constant<bool, true>());
+          else
+            form_p(std::integral_constant<bool, false>());
         }
         // P^T over the group's own first CW/2 S^T columns (already read above)
         FA2_TRACE_AT(trace_row, 58 + g, it);
