@@ -708,6 +708,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
         tc_fence_before();
         mbar_arrive(bar_dq_empty);
+        FA2_TRACE_AT(trace_row, 60 + g, it);
         return true;
       };
       auto drain_st = [&](int it) -> bool {
@@ -727,6 +728,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
               const int row = CW * g + q;
               st_shared_f32(box + row * 128 + ((unit ^ (row & 7)) << 4) + word, dqv[q]);
             }
+            FA2_TRACE_AT(trace_row, 62 + g, it);
             fence_async_smem();
             mbar_arrive(bar_staged);
           } else {
@@ -734,6 +736,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             float* col = acc + static_cast<size_t>(CW * g) * D + r;
 #pragma unroll
             for (int q = 0; q < CW; ++q) red_add(col + static_cast<size_t>(q) * D, dqv[q]);
+            FA2_TRACE_AT(trace_row, 62 + g, it);
           }
         } else {
           if (gg + n > 0 && !mbar_wait(bar_stg_free, (gg + n - 1) & 1, abort_flag, 0x1306)) return false;
