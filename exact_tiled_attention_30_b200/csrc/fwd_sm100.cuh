@@ -643,7 +643,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         // that the P V product actually uses (for O / l, so O stays a convex
         // combination of V rows even when one weight dominates)
         const unsigned long long c2 = f2(c, c), negm2 = f2(-m, -m);
-        unsigned long long rs2 = f2(0.f, 0.f), rr2 = f2(0.f, 0.f);
+        unsigned long long rs2 = f2(0.f, 0.f);
+        float rr_lo = 0.f, rr_hi = 0.f;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           uint32_t pk[16];
@@ -662,7 +663,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               const uint32_t w = pack_bf16(p0, p1);
               pk[i] = w;
               rs2 = f2_add(rs2, f2(p0, p1));
-              rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+              add_bf16x2(rr_lo, rr_hi, w);
             }
           } else {
             // masked keys get exponent -inf, hence weight exactly 0 (also when
@@ -678,7 +679,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               const uint32_t w = pack_bf16(p0, p1);
               pk[i] = w;
               rs2 = f2_add(rs2, f2(p0, p1));
-              rr2 = f2_add(rr2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+              add_bf16x2(rr_lo, rr_hi, w);
             }
           }
           // P of keys [32q, 32q+32) of this half -> columns [16q, 16q+16): the scores
@@ -687,9 +688,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
         FA2_TRACE_AT(trace_row, 8 * t + 3, j);
         FA2_TRACE_AT(trace_last, 8 * t + 6, j);
-        float rs_lo, rs_hi, rr_lo, rr_hi;
+        float rs_lo, rs_hi;
         f2_split(rs2, rs_lo, rs_hi);
-        f2_split(rr2, rr_lo, rr_hi);
         l = l * alpha + (rs_lo + rs_hi);
         lr = lr * alpha + (rr_lo + rr_hi);
         // O must hold PV_0..PV_{j-1} complete. d = 128: it does, since S_j was

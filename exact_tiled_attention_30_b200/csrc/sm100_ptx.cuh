@@ -549,6 +549,16 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` in the low half.
+// lo_acc += low bf16 half of w, hi_acc += high half (each widened exactly to
+// fp32, then one fp32 add with round-to-nearest: the same arithmetic as adding
+// the unpacked values, in one instruction per half)
+__device__ __forceinline__ void add_bf16x2(float& lo_acc, float& hi_acc, uint32_t w) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+      : "+f"(lo_acc), "+f"(hi_acc)
+      : "r"(w));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
