@@ -34,8 +34,8 @@ struct BwdPreParams {
   const __nv_bfloat16* dout;
   const float* lse;
   float* dq_acc;   // [BH][Np][d]
-  float* delta;    // [BH][Np]
-  float* lse2;     // [BH][Np]
+  float* delta;    // [BH][Np]: -D (negated, so the kernels add it)
+  float* lse2;     // [BH][Np]: -LSE * log2 e (negated likewise)
   unsigned int* counter;  // work-item counter of the main kernel
   int N;
   int Np;
@@ -73,9 +73,9 @@ __global__ void __launch_bounds__(256) fa2_bwd_pre_kernel(const BwdPreParams p) 
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (sub == 0) {
-      p.delta[r] = acc;
-      p.lse2[r] = (n < p.N) ? p.lse[static_cast<size_t>(bh) * p.N + n] * 1.4426950408889634f
-                            : INFINITY;
+      p.delta[r] = -acc;
+      p.lse2[r] = (n < p.N) ? p.lse[static_cast<size_t>(bh) * p.N + n] * -1.4426950408889634f
+                            : -INFINITY;
     }
   }
 }
@@ -759,8 +759,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const int i = i_first + it;
         const int gg = gs + it;
         const int s = gg % C::STAGES;
-        const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 2 * C::VEC_BYTES) + CW * g;
-        const float* dlt = lse2 + 128;
+        // -LSE2 and -D of this step's query columns (stored negated, so they add)
+        const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 2 * C::VEC_BYTES) + CW * g;
+        const float* ndlt = nlse2 + 128;
         FA2_TRACE_AT(trace_row, 8 * g + 0, it);
         // LSE2 and D of this query block were written by the TMA (async proxy)
         ok = mbar_wait(bar_st_full(s), (gg / C::STAGES) & 1, abort_flag, 0x1300);
@@ -786,11 +787,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           auto form_p = [&](auto masked) {
 #pragma unroll
             for (int e = 0; e < CW; e += 4) {
-              const float4 l4 = make_float4(lds_f32(lse2 + e), lds_f32(lse2 + e + 1), lds_f32(lse2 + e + 2),
-                                            lds_f32(lse2 + e + 3));
+              const float4 l4 = make_float4(lds_f32(nlse2 + e), lds_f32(nlse2 + e + 1), lds_f32(nlse2 + e + 2),
+                                            lds_f32(nlse2 + e + 3));
               float x0, x1, x2, x3;
-              f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(-l4.x, -l4.y)), x0, x1);
-              f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(-l4.z, -l4.w)), x2, x3);
+              f2_split(f2_fma(f2(sv[e], sv[e + 1]), c2, f2(l4.x, l4.y)), x0, x1);
+              f2_split(f2_fma(f2(sv[e + 2], sv[e + 3]), c2, f2(l4.z, l4.w)), x2, x3);
               float p0, p1, p2, p3;
               if (e / 4 < C::POLY_GROUPS) {  // FMA pipe: takes load off the MUFU unit
                 exp2_poly2(x0, x1, p0, p1);
@@ -841,12 +842,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           tmem_ld32(lane_base + C::COL_DP + CW * g, dp);
 #pragma unroll
           for (int e = 0; e < CW; e += 4) {
-            const float4 d4 = make_float4(lds_f32(dlt + e), lds_f32(dlt + e + 1), lds_f32(dlt + e + 2),
-                                          lds_f32(dlt + e + 3));
+            const float4 d4 = make_float4(lds_f32(ndlt + e), lds_f32(ndlt + e + 1), lds_f32(ndlt + e + 2),
+                                          lds_f32(ndlt + e + 3));
             const unsigned long long pa = f2(__uint_as_float(pk[e / 2] << 16), __uint_as_float(pk[e / 2] & 0xFFFF0000u));
             const unsigned long long pb = f2(__uint_as_float(pk[e / 2 + 1] << 16), __uint_as_float(pk[e / 2 + 1] & 0xFFFF0000u));
-            const unsigned long long da = f2_add(f2(dp[e], dp[e + 1]), f2(-d4.x, -d4.y));
-            const unsigned long long db = f2_add(f2(dp[e + 2], dp[e + 3]), f2(-d4.z, -d4.w));
+            const unsigned long long da = f2_add(f2(dp[e], dp[e + 1]), f2(d4.x, d4.y));
+            const unsigned long long db = f2_add(f2(dp[e + 2], dp[e + 3]), f2(d4.z, d4.w));
             float s0, s1, s2, s3;
             f2_split(f2_mul(pa, da), s0, s1);
             f2_split(f2_mul(pb, db), s2, s3);
@@ -1148,11 +1149,11 @@ __global__ void __launch_bounds__(BwdDqCfg<D>::THREADS, 1)
     const int qrow = qtile * C::BM + r;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const size_t vrow = static_cast<size_t>(bh) * p.Np + qrow;
-    const float lse2 = p.lse2[vrow];   // +inf on padding rows: P = 0 there
-    const float dlt = p.delta[vrow];
+    const float nlse2 = p.lse2[vrow];   // -LSE log2 e; -inf on padding rows: P = 0 there
+    const float ndlt = p.delta[vrow];   // -D
     const unsigned long long c2 = f2(p.scale_log2, p.scale_log2);
-    const unsigned long long nl2 = f2(-lse2, -lse2);
-    const unsigned long long nd2 = f2(-dlt, -dlt);
+    const unsigned long long nl2 = f2(nlse2, nlse2);
+    const unsigned long long nd2 = f2(ndlt, ndlt);
     uint8_t* ds_base = smem + C::OFF_DS;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
