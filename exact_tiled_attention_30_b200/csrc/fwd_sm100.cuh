@@ -19,8 +19,9 @@
 //                 other warps through a two-slot ring, loads Q0, Q1 once the
 //                 previous item's last S MMA is done, K_j/V_j into a STAGES-deep
 //                 ring that continues across items
-//   warp 17       MMA issuer + TMEM owner, running converged (elect.sync
-//                 inside each MMA picks the lane). Per key tile j it issues
+//   (warps 16 and 17 run converged: the whole warp executes the loop and
+//   elect.sync inside each copy / MMA instruction picks the issuing lane)
+//   warp 17       MMA issuer + TMEM owner. Per key tile j it issues
 //                 PV0_j, S0_{j+1}, PV1_j, S1_{j+1} at d = 128 and PV0_j,
 //                 S1_{j+1}, PV1_j, S0_{j+2} at d = 64 (three rotating S
 //                 buffers), so while one tile's softmax runs the tensor core
@@ -28,7 +29,8 @@
 //                 and O_t += P_t V_j (P from TMEM, V from smem). The single issue
 //                 order also keeps the two tiles' softmax phases apart (measured:
 //                 one issuer per tile let them drift into step and contend for
-//                 the MUFU unit).
+//                 the MUFU unit). Non-causal d = 128 launches (EARLY) may issue
+//                 the next item's first S0 while tile 1 forms its last P.
 //   warps 0-7     softmax of query tile 0, warps 8-15 of query tile 1. Two
 //                 warpgroups per tile split each row: warpgroup h owns keys
 //                 [64h, 64h+64) of row r (TMEM lane r): tcgen05.ld of its 64
