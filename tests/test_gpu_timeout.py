@@ -51,7 +51,7 @@ def test_shipped_library_has_no_test_hooks():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("d,causal", [(64, False), (128, True)])
+@pytest.mark.parametrize("d,causal", [(64, False), (128, True), (128, False)])
 def test_stalled_wait_times_out_then_context_recovers(oracle_mod, d, causal):
     import torch
 
