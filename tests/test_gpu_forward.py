@@ -56,6 +56,12 @@ SMALL = [
     (15, 1, 3, 1000, 128, True),
     (16, 2, 3, 384, 128, True),  # several tiles, multiple of 128
     (16, 2, 3, 384, 64, False),
+    # several items per CTA (the persistent grid has one CTA per SM), ragged N:
+    # item boundaries inside a CTA, the non-causal d = 128 early start of the
+    # next item included (one key tile per item at N = 100)
+    (17, 4, 80, 300, 128, False),
+    (17, 4, 80, 300, 64, False),
+    (18, 2, 100, 100, 128, False),
 ]
 
 
