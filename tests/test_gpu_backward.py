@@ -63,6 +63,8 @@ SMALL = [
     (16, 2, 3, 384, 128, True),
     (16, 2, 3, 384, 64, True),
     (16, 2, 3, 384, 128, False),
+    (17, 4, 80, 300, 128, True),  # several items per CTA, ragged N
+    (17, 4, 80, 300, 64, False),
 ]
 
 
